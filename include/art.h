@@ -1,0 +1,168 @@
+/*
+ * art.h -- C ABI of libart, B200 (sm_100a) ART run-time-terminated decode
+ * attention.
+ *
+ * Method: "ART: Attention Run-time Termination for Efficient Large Language
+ * Model Decoding" (gist.science explainer), Technical Summary, section 2.
+ * One decode step of one attention layer: each sequence's single query token
+ * attends over its paged K/V cache.  The cache of each (sequence, kv-head)
+ * unit is walked one block (= one page) at a time in a caller-given order
+ * (section 2.4, traversal reordering), keeping an online-softmax state
+ * (section 2.1).  After every block j >= 1 the partial output o_j (the G
+ * query heads of the unit, concatenated) is compared with o_{j-1}:
+ *
+ *     d_scale = | ||o_j|| - ||o_{j-1}|| | / ||o_{j-1}||      stable if < eps_m
+ *     d_dir   = 1 - cos(o_j, o_{j-1})                      stable if < eps_d
+ *
+ * (section 2.2: both must hold).  A patience counter counts consecutive
+ * stable blocks and resets on an unstable one (section 2.3).  The walk stops
+ * after the block that brings the counter to P, once at least min_blocks
+ * blocks were consumed; the first block of the order is always consumed
+ * (section 2.4, attention sinks).  The blocks after the stop are never
+ * fetched from HBM.  eps = 0 disables termination (full attention).
+ *
+ * Conventions for every entry point:
+ *  - Tensors are described by art_tensor_t: a DEVICE pointer owned by the
+ *    caller, an element type, and shape/stride in ELEMENTS.  The library
+ *    never allocates, frees or retains them.
+ *  - Calls are asynchronous on the given stream (NULL = legacy default
+ *    stream): the results are valid once the stream has reached the call.
+ *  - All argument checks happen on the host, before any CUDA call; a failed
+ *    check returns its status and launches nothing.
+ *  - Errors found on the device (an order or page-table entry out of range,
+ *    a sequence longer than max_blocks pages, an expired wait) never trap:
+ *    the affected unit gets stop_block = -1 and, when the caller passes
+ *    device_status, the first such error code is stored there.
+ */
+#ifndef ART_H
+#define ART_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *art_stream_t;   /* a cudaStream_t */
+
+typedef enum {
+    ART_F32 = 0,    /* IEEE binary32                */
+    ART_BF16 = 1,   /* bfloat16                     */
+    ART_I32 = 2     /* int32                        */
+} art_dtype_t;
+
+typedef struct {
+    void *data;          /* device pointer (caller-owned)                    */
+    int32_t dtype;       /* art_dtype_t                                      */
+    int32_t ndim;        /* number of valid entries in shape/stride          */
+    int64_t shape[4];
+    int64_t stride[4];   /* in elements                                      */
+} art_tensor_t;
+
+typedef enum {
+    ART_OK = 0,
+    ART_ERR_NULL = -1,           /* a required pointer is NULL                           */
+    ART_ERR_SHAPE = -2,          /* inconsistent shapes, strides or alignment            */
+    ART_ERR_DTYPE = -3,          /* wrong or mismatched element type                     */
+    ART_ERR_UNSUPPORTED = -4,    /* head dim, page size or group size not compiled       */
+    ART_ERR_PARAM = -5,          /* eps < 0 or NaN, P < 0, min_blocks < 0, bad option    */
+    ART_ERR_LAUNCH = -6,         /* the CUDA runtime refused the launch                  */
+    ART_ERR_DEVICE_TIMEOUT = -7, /* (device_status) a bounded wait expired               */
+    ART_ERR_BAD_INDEX = -8       /* (device_status) order/page entry or length invalid   */
+} art_status_t;
+
+/*
+ * art_decode_attention -- one ART decode-attention step.
+ *
+ *  q           [B, Hq, d]                     F32 or BF16; d contiguous.
+ *  k_cache     [num_pages, Hkv, page, d]      same type as q; d contiguous; the other
+ *                                             strides multiples of 16 bytes, base 16-byte
+ *                                             aligned (the cache is read with TMA).
+ *  v_cache     same shape and type as k_cache (strides may differ).
+ *  page_table  [B, max_blocks] I32: physical page of logical block lb of sequence b.
+ *  block_order [B, max_blocks] I32: logical block visited at walk step j; entries
+ *                                   0..N_b-1 must be a permutation of 0..N_b-1 where
+ *                                   N_b = ceil(seq_lens[b] / page).  Entries past
+ *                                   N_b are never read.
+ *  seq_lens    [B] I32 (contiguous): tokens in the cache of sequence b.  Token
+ *                                   lb*page + t of the sequence is row t of page
+ *                                   page_table[b, lb]; rows past seq_lens[b] are masked.
+ *  eps_m, eps_d  thresholds (>= 0, not NaN; 0 disables, +inf always passes).
+ *  P           patience (>= 0).  min_blocks: lower bound on blocks consumed (>= 0).
+ *  out         [B, Hq, d] F32: attention output at the stop (0 for empty sequences).
+ *  stop_block  [B, Hkv] I32: blocks consumed by the walk (0 for empty sequences,
+ *                            -1 for a unit that hit a device-side error).
+ * Query head i uses kv head i / (Hq / Hkv).  The softmax scale is 1/sqrt(d).
+ * Supported: d in {64, 128}; page in {16, 64}; Hq/Hkv in 1..8.
+ */
+art_status_t art_decode_attention(const art_tensor_t *q, const art_tensor_t *k_cache,
+                                  const art_tensor_t *v_cache, const art_tensor_t *page_table,
+                                  const art_tensor_t *block_order, const art_tensor_t *seq_lens,
+                                  float eps_m, float eps_d, int32_t P, int32_t min_blocks,
+                                  art_tensor_t *out, art_tensor_t *stop_block, art_stream_t stream);
+
+/* What art_decode_attention_ex chose; filled when art_params_t.info != NULL. */
+typedef struct {
+    int32_t engine;        /* 1 = CUDA-core block engine, 2 = tensor-core (mma) engine   */
+    int32_t cluster_size;  /* CTAs cooperating on one (sequence, kv-head) unit           */
+    int32_t grid;          /* CTAs launched                                               */
+    int32_t threads;       /* threads per CTA                                             */
+    int32_t stages;        /* K/V pages buffered per CTA                                  */
+    int32_t compute_warps; /* warps turning pages into block states, per CTA              */
+    int32_t window;        /* blocks the walk may fetch ahead of the stop decision        */
+    int32_t smem_bytes;    /* dynamic shared memory per CTA                               */
+} art_launch_info_t;
+
+typedef struct {
+    art_tensor_t q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block;
+    float eps_m, eps_d;            /* used where the per-sequence arrays are NULL           */
+    int32_t P, min_blocks;
+    float sm_scale;                /* softmax scale; <= 0 selects 1/sqrt(d)                 */
+    const float *eps_m_per_seq;    /* device [B] or NULL                                    */
+    const float *eps_d_per_seq;    /* device [B] or NULL                                    */
+    const int32_t *P_per_seq;      /* device [B] or NULL                                    */
+    const int32_t *min_blocks_per_seq; /* device [B] or NULL                                */
+    int32_t *blocks_fetched;       /* device [B*Hkv] or NULL: pages whose fetch was issued  */
+    int32_t *device_status;        /* device [1] or NULL: first device-side error (0 = ok); */
+                                   /* the caller zeroes it; the library only writes errors  */
+    int32_t engine;                /* 0 auto, 1 CUDA cores (any dtype), 2 tensor cores (BF16)*/
+    int32_t cluster_size;          /* 0 auto, else 1..16 CTAs per unit                      */
+    int32_t stages;                /* 0 auto, else 2..8 (a multiple of compute_warps)       */
+    int32_t compute_warps;         /* 0 auto, else 1..8                                     */
+    int32_t window;                /* 0 auto, else 2..64 blocks of speculation              */
+    int64_t timeout_ns;            /* 0 = 2 s; bound on every device-side wait              */
+    int32_t debug_flags;           /* 0; bit 0 makes the stop decision wait on a barrier    */
+                                   /* nothing arrives on (exercises the bounded wait)       */
+    art_launch_info_t *info;       /* host pointer or NULL                                  */
+} art_params_t;
+
+/*
+ * art_decode_attention_ex -- the same step with per-sequence thresholds,
+ * an explicit softmax scale, fetch accounting, device status, and launch
+ * overrides.  Passing zeros for every option reproduces art_decode_attention.
+ */
+art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream);
+
+/*
+ * art_build_order_sink_recency -- write the default walk order: for each
+ * sequence b with N_b = ceil(seq_lens[b] / page) blocks, block_order[b] =
+ * [0, N_b-1, N_b-2, ..., 1] followed by -1 up to max_blocks (the sink block
+ * first, then newest to oldest: section 2.4's "recency-first" traversal with
+ * the mandatory block 0).  seq_lens: [B] I32; block_order: [B, max_blocks] I32
+ * with a contiguous last dimension.  A sequence longer than max_blocks pages
+ * gets only its first max_blocks entries (the attention call then reports it).
+ */
+art_status_t art_build_order_sink_recency(const art_tensor_t *seq_lens, int32_t page,
+                                          art_tensor_t *block_order, art_stream_t stream);
+
+/* Static description of a status code. */
+const char *art_strerror(art_status_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t art_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ART_H */

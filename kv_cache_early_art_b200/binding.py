@@ -1,0 +1,194 @@
+"""ctypes binding of libart (include/art.h): argument marshalling only.
+
+Every step of the attention walk runs in the CUDA library; this module turns
+torch tensors into ``art_tensor_t`` descriptors, passes the current CUDA
+stream, and raises ``ArtError`` on a non-zero status.  There is no CPU
+fallback: importing fails when ``libart.so`` has not been built, and calls
+with tensors that are not on a CUDA device are refused.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libart.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libart.so is not built ({LIB_PATH}); run `python -m kv_cache_early_art_b200.build` "
+                      "or __graft_entry__.build()")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+F32, BF16, I32 = 0, 1, 2
+_DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.int32: I32}
+
+STATUS = {
+    0: "ART_OK", -1: "ART_ERR_NULL", -2: "ART_ERR_SHAPE", -3: "ART_ERR_DTYPE", -4: "ART_ERR_UNSUPPORTED",
+    -5: "ART_ERR_PARAM", -6: "ART_ERR_LAUNCH", -7: "ART_ERR_DEVICE_TIMEOUT", -8: "ART_ERR_BAD_INDEX",
+}
+ENGINE_AUTO, ENGINE_CUDA, ENGINE_MMA = 0, 1, 2
+
+
+class ArtTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class ArtLaunchInfo(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("engine", "cluster_size", "grid", "threads", "stages",
+                                               "compute_warps", "window", "smem_bytes")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class ArtParams(ctypes.Structure):
+    _fields_ = [(n, ArtTensor) for n in ("q", "k_cache", "v_cache", "page_table", "block_order", "seq_lens",
+                                         "out", "stop_block")] + [
+        ("eps_m", ctypes.c_float), ("eps_d", ctypes.c_float), ("P", ctypes.c_int32),
+        ("min_blocks", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+        ("eps_m_per_seq", ctypes.c_void_p), ("eps_d_per_seq", ctypes.c_void_p),
+        ("P_per_seq", ctypes.c_void_p), ("min_blocks_per_seq", ctypes.c_void_p),
+        ("blocks_fetched", ctypes.c_void_p), ("device_status", ctypes.c_void_p),
+        ("engine", ctypes.c_int32), ("cluster_size", ctypes.c_int32), ("stages", ctypes.c_int32),
+        ("compute_warps", ctypes.c_int32), ("window", ctypes.c_int32), ("timeout_ns", ctypes.c_int64),
+        ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo))]
+
+
+_P = ctypes.POINTER
+_lib.art_decode_attention.argtypes = [_P(ArtTensor)] * 6 + [ctypes.c_float, ctypes.c_float, ctypes.c_int32,
+                                                            ctypes.c_int32, _P(ArtTensor), _P(ArtTensor),
+                                                            ctypes.c_void_p]
+_lib.art_decode_attention.restype = ctypes.c_int
+_lib.art_decode_attention_ex.argtypes = [_P(ArtParams), ctypes.c_void_p]
+_lib.art_decode_attention_ex.restype = ctypes.c_int
+_lib.art_build_order_sink_recency.argtypes = [_P(ArtTensor), ctypes.c_int32, _P(ArtTensor), ctypes.c_void_p]
+_lib.art_build_order_sink_recency.restype = ctypes.c_int
+_lib.art_strerror.argtypes = [ctypes.c_int]
+_lib.art_strerror.restype = ctypes.c_char_p
+_lib.art_version.argtypes = []
+_lib.art_version.restype = ctypes.c_int32
+
+
+class ArtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({art_strerror(status)})")
+
+
+def art_strerror(status: int) -> str:
+    return _lib.art_strerror(int(status)).decode()
+
+
+def art_version() -> int:
+    return int(_lib.art_version())
+
+
+def descriptor(t: torch.Tensor) -> ArtTensor:
+    """art_tensor_t over a tensor's storage (no copy)."""
+    d = ArtTensor()
+    d.data = t.data_ptr() if t.numel() else None
+    d.dtype = _DTYPE.get(t.dtype, -1)
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libart runs on the GPU only: every tensor must be on a CUDA device")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise ArtError(status, where)
+
+
+def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens, eps_m, eps_d, P, min_blocks,
+                         out=None, stop_block=None, stream=None):
+    """One ART decode-attention step (art_decode_attention in art.h).
+    Returns (out [B,Hq,d] fp32, stop_block [B,Hkv] int32)."""
+    _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    ds = [descriptor(t) for t in (q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)]
+    st = _lib.art_decode_attention(*[ctypes.byref(x) for x in ds[:6]], float(eps_m), float(eps_d), int(P),
+                                   int(min_blocks), ctypes.byref(ds[6]), ctypes.byref(ds[7]), _stream(stream))
+    _check(st, "art_decode_attention")
+    return out, stop_block
+
+
+def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_lens, *, eps_m=0.0, eps_d=0.0,
+                            P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
+                            P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
+                            engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
+                            debug_flags=0, out=None, stop_block=None, stream=None, want_info=False):
+    """art_decode_attention_ex in art.h.  Per-sequence arrays are device
+    tensors of length B (float32 thresholds, int32 P / min_blocks).
+    Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
+    per = [eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status]
+    _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, *per)
+    for t, dt in zip(per, (torch.float32, torch.float32, torch.int32, torch.int32, torch.int32, torch.int32)):
+        if t is not None and (t.dtype != dt or not t.is_contiguous()):
+            raise ValueError(f"per-sequence/accounting arrays must be contiguous {dt}")
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    p = ArtParams()
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("page_table", page_table),
+                    ("block_order", block_order), ("seq_lens", seq_lens), ("out", out), ("stop_block", stop_block)):
+        setattr(p, name, descriptor(t))
+    p.eps_m, p.eps_d, p.P, p.min_blocks = float(eps_m), float(eps_d), int(P), int(min_blocks)
+    p.sm_scale = float(sm_scale)
+    p.eps_m_per_seq = eps_m_per_seq.data_ptr() if eps_m_per_seq is not None else None
+    p.eps_d_per_seq = eps_d_per_seq.data_ptr() if eps_d_per_seq is not None else None
+    p.P_per_seq = P_per_seq.data_ptr() if P_per_seq is not None else None
+    p.min_blocks_per_seq = min_blocks_per_seq.data_ptr() if min_blocks_per_seq is not None else None
+    p.blocks_fetched = blocks_fetched.data_ptr() if blocks_fetched is not None else None
+    p.device_status = device_status.data_ptr() if device_status is not None else None
+    p.engine, p.cluster_size, p.stages = int(engine), int(cluster_size), int(stages)
+    p.compute_warps, p.window, p.timeout_ns = int(compute_warps), int(window), int(timeout_ns)
+    p.debug_flags = int(debug_flags)
+    info = ArtLaunchInfo()
+    p.info = ctypes.pointer(info)
+    st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
+    _check(st, "art_decode_attention_ex")
+    if want_info:
+        return out, stop_block, info.as_dict()
+    return out, stop_block
+
+
+def art_build_order_sink_recency(seq_lens, page, block_order=None, max_blocks=None, stream=None):
+    """Default walk order [0, N-1, ..., 1] (-1 padded) on the device."""
+    _need_cuda(seq_lens, block_order)
+    if block_order is None:
+        if max_blocks is None:
+            raise ValueError("give block_order or max_blocks")
+        block_order = torch.empty(seq_lens.shape[0], int(max_blocks), dtype=torch.int32, device=seq_lens.device)
+    a, b = descriptor(seq_lens), descriptor(block_order)
+    st = _lib.art_build_order_sink_recency(ctypes.byref(a), int(page), ctypes.byref(b), _stream(stream))
+    _check(st, "art_build_order_sink_recency")
+    return block_order
+
+
+def raw_library():
+    """The loaded ctypes library (for ABI tests)."""
+    return _lib

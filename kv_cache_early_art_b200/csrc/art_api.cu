@@ -1,0 +1,514 @@
+// art_api.cu -- host side of libart: argument checks, TMA descriptors, launch
+// shape selection and the extern "C" entry points declared in include/art.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+#include <unordered_map>
+
+#include "../../include/art.h"
+#include "art_kernels.cuh"
+
+namespace {
+
+using art::KernelArgs;
+using art::Layout;
+
+// ---------------------------------------------------------------- checks ----
+
+bool is_null(const art_tensor_t *t) { return t == nullptr || t->data == nullptr; }
+
+int64_t elem_size(int32_t dt) { return dt == ART_BF16 ? 2 : 4; }
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Problem {
+    int dtype;
+    int B, Hq, Hkv, G, d, page, max_blocks, num_pages;
+};
+
+art_status_t check_tensors(const art_params_t *p, Problem *pr)
+{
+    const art_tensor_t *q = &p->q, *k = &p->k_cache, *v = &p->v_cache, *pt = &p->page_table,
+                       *bo = &p->block_order, *sl = &p->seq_lens, *o = &p->out, *st = &p->stop_block;
+    if (is_null(q) || is_null(k) || is_null(v) || is_null(pt) || is_null(bo) || is_null(sl) || is_null(o) ||
+        is_null(st))
+        return ART_ERR_NULL;
+    if (q->ndim != 3 || k->ndim != 4 || v->ndim != 4 || pt->ndim != 2 || bo->ndim != 2 || sl->ndim != 1 ||
+        o->ndim != 3 || st->ndim != 2)
+        return ART_ERR_SHAPE;
+    if (q->dtype != ART_F32 && q->dtype != ART_BF16)
+        return ART_ERR_DTYPE;
+    if (k->dtype != q->dtype || v->dtype != q->dtype || pt->dtype != ART_I32 || bo->dtype != ART_I32 ||
+        sl->dtype != ART_I32 || o->dtype != ART_F32 || st->dtype != ART_I32)
+        return ART_ERR_DTYPE;
+    const int64_t B = q->shape[0], Hq = q->shape[1], d = q->shape[2];
+    const int64_t NP = k->shape[0], Hkv = k->shape[1], page = k->shape[2];
+    if (B <= 0 || Hq <= 0 || d <= 0 || NP <= 0 || Hkv <= 0 || page <= 0)
+        return ART_ERR_SHAPE;
+    if (B > (1 << 24) || Hq > 4096 || NP > (int64_t)INT32_MAX || Hkv > 4096)
+        return ART_ERR_SHAPE;
+    for (int i = 0; i < 4; ++i)
+        if (v->shape[i] != k->shape[i])
+            return ART_ERR_SHAPE;
+    if (k->shape[3] != d || Hq % Hkv != 0)
+        return ART_ERR_SHAPE;
+    if (pt->shape[0] != B || bo->shape[0] != B || pt->shape[1] != bo->shape[1] || pt->shape[1] <= 0 ||
+        pt->shape[1] > (int64_t)INT32_MAX / 256 || sl->shape[0] != B)
+        return ART_ERR_SHAPE;
+    if (o->shape[0] != B || o->shape[1] != Hq || o->shape[2] != d || st->shape[0] != B || st->shape[1] != Hkv)
+        return ART_ERR_SHAPE;
+    // contiguity and alignment the kernels rely on
+    const int64_t es = elem_size(q->dtype);
+    if (q->stride[2] != 1 || k->stride[3] != 1 || v->stride[3] != 1 || pt->stride[1] != 1 ||
+        bo->stride[1] != 1 || sl->stride[0] != 1 || o->stride[2] != 1)
+        return ART_ERR_SHAPE;
+    if (!aligned(q->data, 16) || (q->stride[0] * es) % 16 || (q->stride[1] * es) % 16 || q->stride[0] < 0 ||
+        q->stride[1] < 0)
+        return ART_ERR_SHAPE;
+    for (const art_tensor_t *c : {k, v}) {
+        if (!aligned(c->data, 16))
+            return ART_ERR_SHAPE;
+        for (int i = 0; i < 3; ++i)
+            if (c->stride[i] <= 0 || (c->stride[i] * es) % 16 || c->stride[i] * es >= (int64_t)1 << 40)
+                return ART_ERR_SHAPE;
+    }
+    if (!aligned(pt->data, 4) || !aligned(bo->data, 4) || !aligned(sl->data, 4) || !aligned(o->data, 4) ||
+        !aligned(st->data, 4))
+        return ART_ERR_SHAPE;
+    const int64_t G = Hq / Hkv;
+    if (!(d == 64 || d == 128) || !(page == 16 || page == 64) || G > 8)
+        return ART_ERR_UNSUPPORTED;
+    pr->dtype = q->dtype;
+    pr->B = (int)B;
+    pr->Hq = (int)Hq;
+    pr->Hkv = (int)Hkv;
+    pr->G = (int)G;
+    pr->d = (int)d;
+    pr->page = (int)page;
+    pr->max_blocks = (int)pt->shape[1];
+    pr->num_pages = (int)NP;
+    if ((int64_t)B * Hkv > (int64_t)INT32_MAX / 16)
+        return ART_ERR_SHAPE;
+    return ART_OK;
+}
+
+art_status_t check_params(const art_params_t *p)
+{
+    if (std::isnan(p->eps_m) || std::isnan(p->eps_d) || p->eps_m < 0.f || p->eps_d < 0.f || p->P < 0 ||
+        p->min_blocks < 0)
+        return ART_ERR_PARAM;
+    if (std::isnan(p->sm_scale) || std::isinf(p->sm_scale))
+        return ART_ERR_PARAM;
+    if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
+        p->stages > 8 || p->compute_warps < 0 || p->compute_warps > 8 || p->window < 0 || p->window > 64 ||
+        p->timeout_ns < 0 || (p->debug_flags & ~1))
+        return ART_ERR_PARAM;
+    if (p->stages == 1 || p->window == 1)
+        return ART_ERR_PARAM;
+    for (const void *ptr : {(const void *)p->eps_m_per_seq, (const void *)p->eps_d_per_seq,
+                            (const void *)p->P_per_seq, (const void *)p->min_blocks_per_seq,
+                            (const void *)p->blocks_fetched, (const void *)p->device_status})
+        if (ptr && !aligned(ptr, 4))
+            return ART_ERR_SHAPE;
+    return ART_OK;
+}
+
+// ------------------------------------------------------------- kernels ----
+
+using KernelFn = void (*)(KernelArgs, CUtensorMap, CUtensorMap);
+
+template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+KernelFn kfn()
+{
+    return art::art_walk_kernel<T, D, PAGE, GMAX, ENGINE>;
+}
+
+template <typename T, int ENGINE, int GMAX>
+KernelFn pick_dp(int d, int page)
+{
+    if (d == 64)
+        return page == 16 ? kfn<T, 64, 16, GMAX, ENGINE>() : kfn<T, 64, 64, GMAX, ENGINE>();
+    return page == 16 ? kfn<T, 128, 16, GMAX, ENGINE>() : kfn<T, 128, 64, GMAX, ENGINE>();
+}
+
+int gmax_for(int G, int engine)
+{
+    if (engine == art::kEngineMma)
+        return G <= 4 ? 4 : 8;
+    return G <= 1 ? 1 : (G <= 4 ? 4 : 8);
+}
+
+KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax)
+{
+    if (dtype == ART_F32) {
+        if (gmax == 1) return pick_dp<float, art::kEngineCuda, 1>(d, page);
+        if (gmax == 4) return pick_dp<float, art::kEngineCuda, 4>(d, page);
+        return pick_dp<float, art::kEngineCuda, 8>(d, page);
+    }
+    if (engine == art::kEngineMma) {
+        if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineMma, 4>(d, page);
+        return pick_dp<__nv_bfloat16, art::kEngineMma, 8>(d, page);
+    }
+    if (gmax == 1) return pick_dp<__nv_bfloat16, art::kEngineCuda, 1>(d, page);
+    if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineCuda, 4>(d, page);
+    return pick_dp<__nv_bfloat16, art::kEngineCuda, 8>(d, page);
+}
+
+// ------------------------------------------------------ device caches ----
+
+struct DeviceInfo {
+    int sms = 0, smem_optin = 0;
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceInfo> g_dev;
+std::unordered_map<const void *, int> g_smem_set;   // kernel -> dynamic smem limit already set
+
+art_status_t device_info(DeviceInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return ART_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        DeviceInfo di;
+        if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return ART_ERR_LAUNCH;
+        it = g_dev.emplace(dev, di).first;
+    }
+    *out = it->second;
+    return ART_OK;
+}
+
+art_status_t prepare_kernel(KernelFn fn, int smem)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_smem_set.find((const void *)fn);
+    if (it != g_smem_set.end() && it->second >= smem)
+        return ART_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return ART_ERR_LAUNCH;
+    g_smem_set[(const void *)fn] = smem;
+    return ART_OK;
+}
+
+// ---------------------------------------------------------- tensor maps ----
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 4-D view [num_pages, Hkv, page, d] of a cache; box = one page of one head
+// (d columns, or 64-column slabs with the 128-byte swizzle for the MMA engine).
+art_status_t make_cache_map(CUtensorMap *map, const art_tensor_t *c, int dtype, bool swizzle)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return ART_ERR_LAUNCH;
+    const int64_t es = elem_size(dtype);
+    cuuint64_t dims[4] = {(cuuint64_t)c->shape[3], (cuuint64_t)c->shape[2], (cuuint64_t)c->shape[1],
+                          (cuuint64_t)c->shape[0]};
+    cuuint64_t strides[3] = {(cuuint64_t)(c->stride[2] * es), (cuuint64_t)(c->stride[1] * es),
+                             (cuuint64_t)(c->stride[0] * es)};
+    cuuint32_t box[4] = {(cuuint32_t)(swizzle ? 64 : c->shape[3]), (cuuint32_t)c->shape[2], 1u, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult r = enc(map, dtype == ART_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           4, c->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ART_OK : ART_ERR_LAUNCH;
+}
+
+// -------------------------------------------------------------- launch ----
+
+struct Shape {
+    int engine, gmax, S, NW, R, C, smem, threads;
+};
+
+int smem_bytes(const Shape &s, const Problem &pr)
+{
+    const Layout L = art::make_layout(s.S, s.NW, s.R, pr.page, pr.d, (int)elem_size(pr.dtype), s.gmax,
+                                      s.engine != art::kEngineMma);
+    return (int)L.total + 1024;  // slack to align the base to 1024 bytes
+}
+
+art_status_t choose_shape(const art_params_t *p, const Problem &pr, const DeviceInfo &di, Shape *out)
+{
+    Shape s;
+    s.engine = p->engine ? p->engine : (pr.dtype == ART_BF16 ? art::kEngineMma : art::kEngineCuda);
+    if (s.engine == art::kEngineMma && pr.dtype != ART_BF16)
+        return ART_ERR_UNSUPPORTED;
+    s.gmax = gmax_for(pr.G, s.engine);
+    s.R = p->window ? p->window : 16;
+    s.C = p->cluster_size;
+    const int tile = pr.page * pr.d * (int)elem_size(pr.dtype);
+    // (compute warps, stages) in order of preference: about four 16 KiB pages
+    // (or more, smaller ones) in flight, fewer when a large tile must fit
+    static const int small_tiles[][2] = {{4, 8}, {4, 4}, {2, 4}, {2, 2}, {1, 2}};
+    static const int large_tiles[][2] = {{4, 4}, {2, 4}, {2, 2}, {1, 2}};
+    const int(*cand)[2] = tile >= 16384 ? large_tiles : small_tiles;
+    const int ncand = tile >= 16384 ? 4 : 5;
+    for (int i = 0; i < ncand; ++i) {
+        const int NW = p->compute_warps ? p->compute_warps : cand[i][0];
+        int S = p->stages ? p->stages : cand[i][1];
+        if (!p->stages && S < NW)
+            S = NW;
+        if (S % NW != 0 || S < NW)
+            return ART_ERR_PARAM;
+        s.NW = NW;
+        s.S = S;
+        s.threads = 32 * (2 + NW);
+        s.smem = smem_bytes(s, pr);
+        if (s.smem <= di.smem_optin) {
+            *out = s;
+            return ART_OK;
+        }
+        if (p->compute_warps && p->stages)
+            break;
+    }
+    return ART_ERR_UNSUPPORTED;
+}
+
+art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const DeviceInfo &di, KernelArgs &ka)
+{
+    const int units = pr.B * pr.Hkv;
+    if (s->C > 0)
+        return ART_OK;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, s->threads, s->smem) != cudaSuccess)
+        return ART_ERR_LAUNCH;
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    const int slots = di.sms * per_sm;
+    int C = slots / units;
+    C = C < 1 ? 1 : (C > 16 ? 16 : C);
+    // the largest cluster size whose clusters all fit at once
+    for (; C > 1; --C) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(units * C);
+        cfg.blockDim = dim3(s->threads);
+        cfg.dynamicSmemBytes = s->smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, (void *)fn, &cfg) == cudaSuccess && nclusters >= units)
+            break;
+        cudaGetLastError();
+    }
+    s->C = C;
+    (void)ka;
+    return ART_OK;
+}
+
+art_status_t launch(const art_params_t *p, art_stream_t stream)
+{
+    Problem pr;
+    art_status_t st = check_tensors(p, &pr);
+    if (st != ART_OK)
+        return st;
+    st = check_params(p);
+    if (st != ART_OK)
+        return st;
+    if (p->engine == art::kEngineMma && pr.dtype != ART_BF16)
+        return ART_ERR_UNSUPPORTED;
+
+    DeviceInfo di;
+    if ((st = device_info(&di)) != ART_OK)
+        return st;
+    Shape s;
+    if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
+        return st;
+    KernelFn fn = pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax);
+    if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
+        return st;
+
+    KernelArgs ka;
+    std::memset(&ka, 0, sizeof ka);
+    ka.q = p->q.data;
+    ka.q_sb = p->q.stride[0];
+    ka.q_sh = p->q.stride[1];
+    ka.out = static_cast<float *>(p->out.data);
+    ka.out_sb = p->out.stride[0];
+    ka.out_sh = p->out.stride[1];
+    ka.stop_block = static_cast<int32_t *>(p->stop_block.data);
+    ka.stop_sb = p->stop_block.stride[0];
+    ka.stop_sh = p->stop_block.stride[1];
+    ka.page_table = static_cast<const int32_t *>(p->page_table.data);
+    ka.pt_sb = p->page_table.stride[0];
+    ka.block_order = static_cast<const int32_t *>(p->block_order.data);
+    ka.bo_sb = p->block_order.stride[0];
+    ka.seq_lens = static_cast<const int32_t *>(p->seq_lens.data);
+    ka.eps_m_arr = p->eps_m_per_seq;
+    ka.eps_d_arr = p->eps_d_per_seq;
+    ka.P_arr = p->P_per_seq;
+    ka.minb_arr = p->min_blocks_per_seq;
+    ka.eps_m = p->eps_m;
+    ka.eps_d = p->eps_d;
+    ka.P = p->P;
+    ka.min_blocks = p->min_blocks;
+    const float scale = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)pr.d);
+    ka.scale_log2 = scale * 1.4426950408889634f;
+    ka.blocks_fetched = p->blocks_fetched;
+    ka.device_status = p->device_status;
+    ka.B = pr.B;
+    ka.Hq = pr.Hq;
+    ka.Hkv = pr.Hkv;
+    ka.G = pr.G;
+    ka.num_pages = pr.num_pages;
+    ka.max_blocks = pr.max_blocks;
+    ka.timeout_ns = p->timeout_ns > 0 ? p->timeout_ns : 2000000000LL;
+    ka.debug_flags = p->debug_flags;
+
+    if ((st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
+        return st;
+    ka.C = s.C;
+    ka.S = s.S;
+    ka.NW = s.NW;
+    ka.R = s.R;
+
+    CUtensorMap tmk, tmv;
+    const bool swz = s.engine == art::kEngineMma;
+    if ((st = make_cache_map(&tmk, &p->k_cache, pr.dtype, swz)) != ART_OK)
+        return st;
+    if ((st = make_cache_map(&tmv, &p->v_cache, pr.dtype, swz)) != ART_OK)
+        return st;
+
+    const int units = pr.B * pr.Hkv;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = s.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(units * s.C);
+    cfg.blockDim = dim3(s.threads);
+    cfg.dynamicSmemBytes = s.smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (p->info) {
+        p->info->engine = s.engine;
+        p->info->cluster_size = s.C;
+        p->info->grid = units * s.C;
+        p->info->threads = s.threads;
+        p->info->stages = s.S;
+        p->info->compute_warps = s.NW;
+        p->info->window = s.R;
+        p->info->smem_bytes = s.smem;
+    }
+    if (cudaLaunchKernelEx(&cfg, fn, ka, tmk, tmv) != cudaSuccess) {
+        cudaGetLastError();
+        return ART_ERR_LAUNCH;
+    }
+    return ART_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
+{
+    if (!p)
+        return ART_ERR_NULL;
+    return launch(p, stream);
+}
+
+art_status_t art_decode_attention(const art_tensor_t *q, const art_tensor_t *k_cache, const art_tensor_t *v_cache,
+                                  const art_tensor_t *page_table, const art_tensor_t *block_order,
+                                  const art_tensor_t *seq_lens, float eps_m, float eps_d, int32_t P,
+                                  int32_t min_blocks, art_tensor_t *out, art_tensor_t *stop_block,
+                                  art_stream_t stream)
+{
+    if (!q || !k_cache || !v_cache || !page_table || !block_order || !seq_lens || !out || !stop_block)
+        return ART_ERR_NULL;
+    art_params_t p;
+    std::memset(&p, 0, sizeof p);
+    p.q = *q;
+    p.k_cache = *k_cache;
+    p.v_cache = *v_cache;
+    p.page_table = *page_table;
+    p.block_order = *block_order;
+    p.seq_lens = *seq_lens;
+    p.out = *out;
+    p.stop_block = *stop_block;
+    p.eps_m = eps_m;
+    p.eps_d = eps_d;
+    p.P = P;
+    p.min_blocks = min_blocks;
+    return launch(&p, stream);
+}
+
+art_status_t art_build_order_sink_recency(const art_tensor_t *seq_lens, int32_t page, art_tensor_t *block_order,
+                                          art_stream_t stream)
+{
+    if (is_null(seq_lens) || is_null(block_order))
+        return ART_ERR_NULL;
+    if (seq_lens->ndim != 1 || block_order->ndim != 2 || seq_lens->dtype != ART_I32 ||
+        block_order->dtype != ART_I32)
+        return seq_lens->ndim != 1 || block_order->ndim != 2 ? ART_ERR_SHAPE : ART_ERR_DTYPE;
+    const int64_t B = seq_lens->shape[0];
+    if (B <= 0 || B > 65535 || block_order->shape[0] != B || block_order->shape[1] <= 0 ||
+        block_order->shape[1] > (int64_t)INT32_MAX || seq_lens->stride[0] != 1 || block_order->stride[1] != 1 ||
+        block_order->stride[0] < block_order->shape[1])
+        return ART_ERR_SHAPE;
+    if (page <= 0)
+        return ART_ERR_PARAM;
+    if (!aligned(seq_lens->data, 4) || !aligned(block_order->data, 4))
+        return ART_ERR_SHAPE;
+    const int mb = (int)block_order->shape[1];
+    const int threads = 256;
+    int gx = (mb + threads - 1) / threads;
+    gx = gx > 64 ? 64 : gx;
+    art::art_build_order_kernel<<<dim3(gx, (unsigned)B), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const int32_t *>(seq_lens->data), (int)B, page, static_cast<int32_t *>(block_order->data),
+        block_order->stride[0], mb);
+    if (cudaGetLastError() != cudaSuccess)
+        return ART_ERR_LAUNCH;
+    return ART_OK;
+}
+
+const char *art_strerror(art_status_t s)
+{
+    switch (s) {
+    case ART_OK: return "success";
+    case ART_ERR_NULL: return "a required pointer is NULL";
+    case ART_ERR_SHAPE: return "inconsistent shapes, strides or alignment";
+    case ART_ERR_DTYPE: return "wrong or mismatched element type";
+    case ART_ERR_UNSUPPORTED: return "head dim, page size or group size not supported";
+    case ART_ERR_PARAM: return "invalid threshold, patience, min_blocks or option";
+    case ART_ERR_LAUNCH: return "the CUDA runtime refused the launch";
+    case ART_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case ART_ERR_BAD_INDEX: return "an order or page-table entry, or a sequence length, is out of range";
+    }
+    return "unknown status";
+}
+
+int32_t art_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,936 @@
+// art_kernels.cuh -- ART run-time-terminated decode attention for sm_100a.
+//
+// Method: "ART: Attention Run-time Termination for Efficient Large Language
+// Model Decoding" (gist.science explainer), Technical Summary section 2:
+// 2.1 streaming tile-wise online-softmax accumulation, 2.2 the magnitude and
+// direction statistics of the partial output and their thresholds, 2.3 the
+// patience counter, 2.4 caller-chosen traversal order with the sink block
+// always consumed.  The exact statistics are the relative magnitude change
+// |‖o_j‖-‖o_{j-1}‖|/‖o_{j-1}‖ < eps_m and 1-cos(o_j,o_{j-1}) < eps_d over the
+// concatenated outputs of the G query heads that share a kv head.
+//
+// Organisation (one cluster of C CTAs per (sequence, kv-head) unit):
+//
+//   producer warp   walks this CTA's share of the order (steps j = rank,
+//                   rank+C, ...), fetches each page's K and V tiles with TMA
+//                   into a ring of S stages, and never runs more than R steps
+//                   ahead of the merged prefix (R = speculation window).  Once
+//                   the stop is known it issues nothing more.
+//   compute warps   turn one staged page into a block-local softmax state
+//                   (m_j, l_j, u_j = P_j V_j / l_j per head), independent of all
+//                   other blocks, and push it into the leader's ring slot j % R.
+//   merge warp      (leader CTA only) folds the block states into the running
+//                   output in walk order: o_j = o_{j-1} + beta_j (u_j - o_{j-1}),
+//                   beta_j the block's share of the softmax mass.  The same pass
+//                   forms the two statistics from Delta_j = o_j - o_{j-1} without
+//                   cancellation, runs the patience rule and publishes the stop.
+//
+// Because every block state is exact on its own and the merge is sequential,
+// the stop index is the one a strictly sequential walk would take; pages
+// fetched past the stop are bounded by the window R.  Every wait is bounded by
+// a timeout that raises an error flag instead of trapping.
+#pragma once
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "art_ptx.cuh"
+
+namespace art {
+
+constexpr uint32_t kStopBit = 0x80000000u;
+constexpr uint32_t kEndOfStream = 0xFFFFFFFFu;
+constexpr int kMaxThreads = 320;  // producer + merge + up to 8 compute warps
+constexpr int kErrTimeout = -7;
+constexpr int kErrBadIndex = -8;
+constexpr int kEngineCuda = 1;
+constexpr int kEngineMma = 2;
+
+struct KernelArgs {
+    const void *q;
+    int64_t q_sb, q_sh;                 // element strides of q (d is contiguous)
+    float *out;
+    int64_t out_sb, out_sh;
+    int32_t *stop_block;
+    int64_t stop_sb, stop_sh;
+    const int32_t *page_table;
+    int64_t pt_sb;
+    const int32_t *block_order;
+    int64_t bo_sb;
+    const int32_t *seq_lens;
+    const float *eps_m_arr, *eps_d_arr;
+    const int32_t *P_arr, *minb_arr;
+    float eps_m, eps_d;
+    int32_t P, min_blocks;
+    float scale_log2;                   // softmax scale * log2(e)
+    int32_t *blocks_fetched;
+    int32_t *device_status;
+    int32_t B, Hq, Hkv, G, num_pages, max_blocks;
+    int32_t C, S, NW, R;                // cluster size, stages, compute warps, window
+    int64_t timeout_ns;
+    int32_t debug_flags;
+};
+
+// Shared-memory carve-up, identical on host and device.
+struct Layout {
+    uint32_t tile_bytes, stage_bytes;
+    uint32_t kv_off, ring_off, slot_bytes, u_off_floats;
+    uint32_t pbuf_off, meta_off, bar_off, ctrl_off, total;
+};
+
+__host__ __device__ inline uint32_t round_up_u32(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline Layout make_layout(int S, int NW, int R, int page, int d, int esize, int gmax,
+                                              bool pbuf)
+{
+    Layout L;
+    L.tile_bytes = (uint32_t)(page * d * esize);
+    L.stage_bytes = 2 * L.tile_bytes;
+    L.kv_off = 0;
+    uint32_t off = S * L.stage_bytes;
+    // slot: [flag, pad x3][m x gmax][l x gmax][pad][u x gmax*d]   (floats)
+    L.u_off_floats = round_up_u32(4 + 2 * gmax, 4);
+    L.slot_bytes = round_up_u32((L.u_off_floats + gmax * d) * 4, 16);
+    L.ring_off = off;
+    off += R * L.slot_bytes;
+    L.pbuf_off = off;
+    off += pbuf ? (uint32_t)(NW * page * gmax * 4) : 0u;
+    L.meta_off = off;
+    off += 2 * S * 4;  // stage_j[S], stage_nv[S]
+    off = round_up_u32(off, 8);
+    L.bar_off = off;
+    off += (3 * S + R + 1) * 8;  // full_k, full_v, empty, ready, never
+    L.ctrl_off = off;
+    off += 16;  // ctrl, fetched, abort, pad
+    L.total = off;
+    return L;
+}
+
+__device__ __forceinline__ void record_error(int32_t *status, int code)
+{
+    if (status)
+        atomicCAS(status, 0, code);
+}
+
+// Warp-wide bounded wait on an mbarrier phase.  Returns false (without
+// trapping) when this CTA was told to abort or when timeout_ns passes; the
+// latter also raises the abort flag and records the timeout.
+template <bool kClusterAcquire>
+__device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int64_t timeout_ns,
+                                       int32_t *status, bool respect_abort = true)
+{
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool ok = kClusterAcquire ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, ok))
+            return true;
+        if ((it & 7u) == 7u) {
+            int quit = 0;
+            if ((threadIdx.x & 31) == 0) {
+                const uint64_t now = global_timer_ns();
+                if (t0 == 0)
+                    t0 = now;
+                if (respect_abort && *abort) {
+                    quit = 1;
+                } else if ((int64_t)(now - t0) > timeout_ns) {
+                    *abort = 1u;
+                    record_error(status, kErrTimeout);
+                    quit = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, quit, 0))
+                return false;
+        }
+    }
+}
+
+// ---- element loads ---------------------------------------------------------
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// DE consecutive elements of a shared-memory row starting at element lane*DE.
+template <typename T, int DE>
+__device__ __forceinline__ void load_chunk(const uint8_t *row, int lane, float (&f)[DE])
+{
+    if constexpr (sizeof(T) == 4) {
+        const float *p = reinterpret_cast<const float *>(row) + lane * DE;
+        if constexpr (DE == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(p);
+            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(p);
+            f[0] = v.x; f[1] = v.y;
+        }
+    } else {
+        const uint8_t *p = row + lane * DE * 2;
+        if constexpr (DE == 4) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(p);
+            f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+        } else {
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(p);
+            f[0] = bf16_lo(v); f[1] = bf16_hi(v);
+        }
+    }
+}
+
+// Butterfly reduce-scatter of 32 per-lane partial sums: afterwards v[0] of
+// lane l holds the warp-wide sum of entry l.
+__device__ __forceinline__ void reduce_scatter32(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+            const float send = upper ? v[i] : v[i + k];
+            const float keep = upper ? v[i + k] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+}
+
+// Byte offset of bf16 element (t, d) in a K or V tile stored as d/64 column
+// slabs of [page][64] with the 128-byte TMA swizzle (16-byte chunk index
+// XOR row mod 8).
+template <int PAGE>
+__device__ __forceinline__ uint32_t swz128(int t, int d)
+{
+    return (uint32_t)((d >> 6) * PAGE * 128 + t * 128 + ((((d & 63) >> 3) ^ (t & 7)) << 4) + (d & 7) * 2);
+}
+
+// ---- shared state handed to the roles ---------------------------------------
+
+struct Shared {
+    uint8_t *kv;          // S stages of [K tile | V tile]
+    float *ring;          // R slots (meaningful in the leader)
+    float *pbuf;          // per compute warp [PAGE][GMAX] (CUDA-core engine)
+    uint32_t *stage_j, *stage_nv;
+    uint32_t bar0;        // shared address of full_k[0]
+    volatile uint32_t *ctrl, *fetched, *abort;
+    Layout L;
+    __device__ uint32_t full_k(int s) const { return bar0 + 8u * s; }
+    __device__ uint32_t full_v(int s, int S) const { return bar0 + 8u * (S + s); }
+    __device__ uint32_t empty(int s, int S) const { return bar0 + 8u * (2 * S + s); }
+    __device__ uint32_t ready(int r, int S) const { return bar0 + 8u * (3 * S + r); }
+    __device__ uint32_t never(int S, int R) const { return bar0 + 8u * (3 * S + R); }
+};
+
+// ---- producer ----------------------------------------------------------------
+
+template <typename T, int D, int PAGE, int ENGINE>
+__device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUtensorMap *tmk, const CUtensorMap *tmv,
+                              int b, int h, int N, int Lseq, uint32_t rank)
+{
+    const int lane = threadIdx.x & 31;
+    const int S = a.S, R = a.R, C = a.C;
+    const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
+    const int32_t *bo = a.block_order + (int64_t)b * a.bo_sb;
+    const int32_t *pt = a.page_table + (int64_t)b * a.pt_sb;
+    if (lane == 0) {
+        prefetch_tensormap(tmk);
+        prefetch_tensormap(tmv);
+    }
+    uint32_t issued = 0;        // stages handed out (pages, markers)
+    uint32_t kphase = 0, vphase = 0;  // bit s: parity of the last phase armed on full_k[s] / full_v[s]
+    uint32_t kused = 0, vused = 0;
+    uint32_t nfetched = 0;
+    int batch_k0 = -1, my_lb = -1, my_pp = -1;
+    bool aborted = false;
+
+    auto take_stage = [&](uint32_t i) -> bool {  // wait until stage i % S is free
+        const int s = (int)(i % (uint32_t)S);
+        if (i < (uint32_t)S)
+            return true;
+        return warp_wait<false>(sh.empty(s, S), ((i / S) - 1) & 1u, sh.abort, a.timeout_ns, a.device_status);
+    };
+
+    for (int k = 0;; ++k) {
+        const int j = (int)rank + k * C;
+        if (j >= N)
+            break;
+        if (batch_k0 < 0 || k - batch_k0 >= 32) {  // fetch the next 32 index pairs at once
+            batch_k0 = k;
+            const int jj = (int)rank + (k + lane) * C;
+            my_lb = -1;
+            my_pp = -1;
+            if (jj < N) {
+                my_lb = __ldg(bo + jj);
+                if (my_lb >= 0 && my_lb < N)
+                    my_pp = __ldg(pt + my_lb);
+            }
+        }
+        const int lb = __shfl_sync(0xffffffffu, my_lb, k - batch_k0);
+        const int pp = __shfl_sync(0xffffffffu, my_pp, k - batch_k0);
+        const bool bad = lb < 0 || lb >= N || pp < 0 || pp >= a.num_pages;
+
+        // speculation window: step j only once j < merged + R
+        int go = 1;
+        if (lane == 0) {
+            uint64_t t0 = 0;
+            for (uint32_t it = 0;; ++it) {
+                const uint32_t c = ld_acquire_cluster_u32(ctrl_cl);
+                if (c & kStopBit) { go = 0; break; }
+                if ((uint32_t)j < c + (uint32_t)R) break;
+                if ((it & 15u) == 15u) {
+                    const uint64_t now = global_timer_ns();
+                    if (t0 == 0) t0 = now;
+                    if (*sh.abort) { go = -1; break; }
+                    if ((int64_t)(now - t0) > a.timeout_ns) {
+                        *sh.abort = 1u;
+                        record_error(a.device_status, kErrTimeout);
+                        go = -1;
+                        break;
+                    }
+                }
+            }
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (go == 0)
+            break;
+        if (go < 0) { aborted = true; break; }
+        if (!take_stage(issued)) { aborted = true; break; }
+        const int s = (int)(issued % (uint32_t)S);
+        if (lane == 0) {
+            sh.stage_j[s] = (uint32_t)j;
+            if (bad) {
+                // pass the fault down the pipeline: the merge reports it
+                sh.stage_nv[s] = 0xFFFFFFFFu;
+                mbar_arrive(sh.full_k(s));
+                mbar_arrive(sh.full_v(s, S));
+                record_error(a.device_status, kErrBadIndex);
+            } else {
+                const int nv = min(PAGE, Lseq - lb * PAGE);
+                sh.stage_nv[s] = (uint32_t)nv;
+                const uint32_t kdst = smem_u32(sh.kv + (size_t)s * sh.L.stage_bytes);
+                const uint32_t vdst = kdst + sh.L.tile_bytes;
+                mbar_arrive_expect_tx(sh.full_k(s), sh.L.tile_bytes);
+                if constexpr (ENGINE == kEngineMma) {
+#pragma unroll
+                    for (int sb = 0; sb < D / 64; ++sb)
+                        tma_load_4d(kdst + sb * PAGE * 128, tmk, sb * 64, 0, h, pp, sh.full_k(s));
+                } else {
+                    tma_load_4d(kdst, tmk, 0, 0, h, pp, sh.full_k(s));
+                }
+                mbar_arrive_expect_tx(sh.full_v(s, S), sh.L.tile_bytes);
+                if constexpr (ENGINE == kEngineMma) {
+#pragma unroll
+                    for (int sb = 0; sb < D / 64; ++sb)
+                        tma_load_4d(vdst + sb * PAGE * 128, tmv, sb * 64, 0, h, pp, sh.full_v(s, S));
+                } else {
+                    tma_load_4d(vdst, tmv, 0, 0, h, pp, sh.full_v(s, S));
+                }
+            }
+        }
+        kphase ^= (kused >> s & 1u) ? (1u << s) : 0u;
+        kused |= 1u << s;
+        vphase ^= (vused >> s & 1u) ? (1u << s) : 0u;
+        vused |= 1u << s;
+        ++issued;
+        if (!bad)
+            ++nfetched;
+        else
+            break;
+    }
+
+    if (!aborted) {
+        // one end-of-stream marker per compute warp, in issue order
+        for (int w = 0; w < a.NW; ++w) {
+            if (!take_stage(issued)) { aborted = true; break; }
+            const int s = (int)(issued % (uint32_t)S);
+            if (lane == 0) {
+                sh.stage_j[s] = kEndOfStream;
+                mbar_arrive(sh.full_k(s));
+            }
+            kphase ^= (kused >> s & 1u) ? (1u << s) : 0u;
+            kused |= 1u << s;
+            ++issued;
+        }
+    }
+    if (aborted) {
+        // let every copy already in flight land before shared memory goes away
+        for (int s = 0; s < S; ++s) {
+            if (kused >> s & 1u)
+                warp_wait<false>(sh.full_k(s), kphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
+            if (vused >> s & 1u)
+                warp_wait<false>(sh.full_v(s, S), vphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
+        }
+    }
+    if (lane == 0)
+        atom_add_cluster_u32(mapa(smem_u32((const void *)sh.fetched), 0), nfetched);
+}
+
+// ---- block engines -------------------------------------------------------------
+//
+// Each turns one staged page into (m_g, l_g, u_g) for the G query heads:
+// m_g = max_t s_gt (log2 domain), l_g = sum_t 2^(s_gt - m_g),
+// u_g = sum_t 2^(s_gt - m_g) v_t / l_g, and writes them to the leader's slot.
+
+struct SlotRef {
+    uint32_t base;   // cluster address of the slot
+    uint32_t ready;  // cluster address of its ready barrier
+};
+
+__device__ __forceinline__ void publish_slot_flag(const SlotRef &sr, int lane, uint32_t flag)
+{
+    if (lane == 0)
+        st_cluster_f32(sr.base, __uint_as_float(flag));
+}
+
+// CUDA-core engine: lane l owns head-dim elements [l*DE, l*DE+DE).
+template <typename T, int D, int PAGE, int GMAX>
+struct CudaEngine {
+    static constexpr int DE = D / 32;
+    static constexpr int TB = 32 / GMAX;              // tokens per butterfly batch
+    static constexpr int NB = (PAGE + TB - 1) / TB;   // batches per page
+    float qf[GMAX][DE];
+
+    __device__ void load_q(const KernelArgs &a, int b, int h, int lane)
+    {
+        const T *qp = reinterpret_cast<const T *>(a.q) + (int64_t)b * a.q_sb;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g)
+#pragma unroll
+            for (int e = 0; e < DE; ++e)
+                qf[g][e] = (g < a.G) ? to_f32<T>(qp[(int64_t)(h * a.G + g) * a.q_sh + lane * DE + e]) : 0.f;
+    }
+
+    // returns false on abort
+    __device__ bool block(const KernelArgs &a, const Shared &sh, int s, uint32_t par, int nv, float *pbuf,
+                          const SlotRef &sr, uint32_t u_off, int lane)
+    {
+        const uint8_t *kt = sh.kv + (size_t)s * sh.L.stage_bytes;
+        const uint8_t *vt = kt + sh.L.tile_bytes;
+        constexpr int ROWB = D * (int)sizeof(T);
+        float sc[NB];
+#pragma unroll
+        for (int bt = 0; bt < NB; ++bt) {
+            float v[32];
+#pragma unroll
+            for (int tt = 0; tt < TB; ++tt) {
+                const int t = bt * TB + tt;
+                if (t < PAGE) {
+                    float kf[DE];
+                    load_chunk<T, DE>(kt + t * ROWB, lane, kf);
+#pragma unroll
+                    for (int g = 0; g < GMAX; ++g) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < DE; ++e)
+                            acc = fmaf(qf[g][e], kf[e], acc);
+                        v[tt * GMAX + g] = acc;
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < GMAX; ++g)
+                        v[tt * GMAX + g] = 0.f;
+                }
+            }
+            reduce_scatter32(v, lane);
+            sc[bt] = v[0];
+        }
+        // lane holds the score of token bt*TB + lane/GMAX for head lane%GMAX
+        const int gl = lane % GMAX;
+        float m = -CUDART_INF_F;
+#pragma unroll
+        for (int bt = 0; bt < NB; ++bt) {
+            const int t = bt * TB + lane / GMAX;
+            const bool valid = (t < nv) && (gl < a.G);
+            sc[bt] = valid ? sc[bt] * a.scale_log2 : -CUDART_INF_F;
+            m = fmaxf(m, sc[bt]);
+        }
+#pragma unroll
+        for (int off = 16; off >= GMAX; off >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f;
+#pragma unroll
+        for (int bt = 0; bt < NB; ++bt) {
+            const int t = bt * TB + lane / GMAX;
+            const float p = (sc[bt] == -CUDART_INF_F) ? 0.f : exp2f(sc[bt] - m);
+            l += p;
+            if (t < PAGE)
+                pbuf[t * GMAX + gl] = p;
+        }
+#pragma unroll
+        for (int off = 16; off >= GMAX; off >>= 1)
+            l += __shfl_xor_sync(0xffffffffu, l, off);
+        __syncwarp();
+
+        if (!warp_wait<false>(sh.full_v(s, a.S), par, sh.abort, a.timeout_ns, a.device_status))
+            return false;
+        float acc[GMAX][DE];
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g)
+#pragma unroll
+            for (int e = 0; e < DE; ++e)
+                acc[g][e] = 0.f;
+#pragma unroll 4
+        for (int t = 0; t < nv; ++t) {
+            float vf[DE];
+            load_chunk<T, DE>(vt + t * ROWB, lane, vf);
+            float pg[GMAX];
+#pragma unroll
+            for (int g = 0; g < GMAX; ++g)
+                pg[g] = pbuf[t * GMAX + g];
+#pragma unroll
+            for (int g = 0; g < GMAX; ++g)
+#pragma unroll
+                for (int e = 0; e < DE; ++e)
+                    acc[g][e] = fmaf(pg[g], vf[e], acc[g][e]);
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(sh.empty(s, a.S));
+
+        // block state into the leader's slot
+        if (lane < GMAX && lane < a.G) {
+            st_cluster_f32(sr.base + 4u * (4 + lane), m);
+            st_cluster_f32(sr.base + 4u * (4 + GMAX + lane), l);
+        }
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+            const float lg = __shfl_sync(0xffffffffu, l, g);
+            if (g < a.G) {
+                const float inv = lg > 0.f ? 1.f / lg : 0.f;
+                const uint32_t addr = sr.base + 4u * (u_off + g * D + lane * DE);
+                if constexpr (DE == 4)
+                    st_cluster_v4(addr, acc[g][0] * inv, acc[g][1] * inv, acc[g][2] * inv, acc[g][3] * inv);
+                else
+                    st_cluster_v2(addr, acc[g][0] * inv, acc[g][1] * inv);
+            }
+        }
+        publish_slot_flag(sr, lane, 0u);
+        mbar_arrive_cluster(sr.ready);
+        return true;
+    }
+};
+
+// Tensor-core engine (bf16): S^T = K q^T with mma.m16n8k16 (tokens x heads),
+// then O^T = V^T P^T with P kept to ~16 significant bits as a bf16 hi + lo pair
+// (for G <= 4 both halves share one n8 tile: columns 0-3 hi, 4-7 lo).
+template <int D, int PAGE, int GMAX>
+struct MmaEngine {
+    static constexpr int MT = PAGE / 16;  // token tiles
+    static constexpr int KS = D / 16;     // head-dim tiles
+    static constexpr bool kShared = GMAX <= 4;
+    uint32_t qb[KS][2];
+
+    __device__ void load_q(const KernelArgs &a, int b, int h, int lane)
+    {
+        const int r = lane >> 2, c = lane & 3;
+        const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + (int64_t)b * a.q_sb;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qb[ks][0] = 0u;
+            qb[ks][1] = 0u;
+            if (r < a.G) {
+                const __nv_bfloat16 *row = qp + (int64_t)(h * a.G + r) * a.q_sh + ks * 16 + 2 * c;
+                qb[ks][0] = *reinterpret_cast<const uint32_t *>(row);
+                qb[ks][1] = *reinterpret_cast<const uint32_t *>(row + 8);
+            }
+        }
+    }
+
+    __device__ bool block(const KernelArgs &a, const Shared &sh, int s, uint32_t par, int nv, float *,
+                          const SlotRef &sr, uint32_t u_off, int lane)
+    {
+        const int r = lane >> 2, c = lane & 3;
+        uint8_t *kt = sh.kv + (size_t)s * sh.L.stage_bytes;
+        uint8_t *vt = kt + sh.L.tile_bytes;
+        const uint32_t ku = smem_u32(kt), vu = smem_u32(vt);
+
+        // scores, rows = tokens, columns = heads
+        float sacc[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                const int t = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int d = ks * 16 + (lane >> 4) * 8;
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(ku + swz128<PAGE>(t, d), a0, a1, a2, a3);
+                mma_bf16_16816(sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+            }
+        }
+        const int g0 = 2 * c;
+        float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = mt * 16 + r + (i >> 1) * 8;
+                const bool valid = (t < nv) && (g0 + (i & 1) < a.G);
+                sacc[mt][i] = valid ? sacc[mt][i] * a.scale_log2 : -CUDART_INF_F;
+                m2[i & 1] = fmaxf(m2[i & 1], sacc[mt][i]);
+            }
+#pragma unroll
+        for (int off = 4; off <= 16; off <<= 1) {
+            m2[0] = fmaxf(m2[0], __shfl_xor_sync(0xffffffffu, m2[0], off));
+            m2[1] = fmaxf(m2[1], __shfl_xor_sync(0xffffffffu, m2[1], off));
+        }
+        float l2[2] = {0.f, 0.f};
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float p = (sacc[mt][i] == -CUDART_INF_F) ? 0.f : exp2f(sacc[mt][i] - m2[i & 1]);
+                sacc[mt][i] = p;
+                l2[i & 1] += p;
+            }
+#pragma unroll
+        for (int off = 4; off <= 16; off <<= 1) {
+            l2[0] += __shfl_xor_sync(0xffffffffu, l2[0], off);
+            l2[1] += __shfl_xor_sync(0xffffffffu, l2[1], off);
+        }
+
+        // P as B operands: bh (hi, or hi|lo when shared), bl (lo, G > 4)
+        uint32_t bh[MT][2], bl[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const float p0 = sacc[mt][2 * half], p1 = sacc[mt][2 * half + 1];
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+                const float2 hf = __bfloat1622float2(hi);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                const uint32_t hu = *reinterpret_cast<const uint32_t *>(&hi);
+                const uint32_t lu = *reinterpret_cast<const uint32_t *>(&lo);
+                if constexpr (kShared) {
+                    const uint32_t lo_from = __shfl_xor_sync(0xffffffffu, lu, 2);
+                    bh[mt][half] = movmatrix_trans(c < 2 ? hu : lo_from);
+                    bl[mt][half] = 0u;
+                } else {
+                    bh[mt][half] = movmatrix_trans(hu);
+                    bl[mt][half] = movmatrix_trans(lu);
+                }
+            }
+
+        if (!warp_wait<false>(sh.full_v(s, a.S), par, sh.abort, a.timeout_ns, a.device_status))
+            return false;
+        if (nv < PAGE) {
+            // rows past the sequence end may hold anything: zero them so 0 * x = 0
+            constexpr int CH = D / 64 * 8;  // 16-byte chunks per row
+            for (int idx = lane; idx < (PAGE - nv) * CH; idx += 32) {
+                const int t = nv + idx / CH, ch = idx % CH;
+                *reinterpret_cast<uint4 *>(vt + (ch >> 3) * PAGE * 128 + t * 128 + (ch & 7) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        float oacc[KS][4], oacc2[KS][4];
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                oacc[dt][i] = oacc2[dt][i] = 0.f;
+#pragma unroll
+            for (int kt2 = 0; kt2 < MT; ++kt2) {
+                const int t = kt2 * 16 + (lane & 7) + (lane >> 4) * 8;
+                const int d = dt * 16 + ((lane >> 3) & 1) * 8;
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4_trans(vu + swz128<PAGE>(t, d), a0, a1, a2, a3);
+                mma_bf16_16816(oacc[dt], a0, a1, a2, a3, bh[kt2][0], bh[kt2][1]);
+                if constexpr (!kShared)
+                    mma_bf16_16816(oacc2[dt], a0, a1, a2, a3, bl[kt2][0], bl[kt2][1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(sh.empty(s, a.S));
+
+        // columns of this lane after combining hi and lo: heads gA, gA+1
+        const int gA = kShared ? 2 * (c & 1) : 2 * c;
+        const bool writer = kShared ? (c < 2) : true;
+        float tot[KS][4];
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if constexpr (kShared)
+                    tot[dt][i] = oacc[dt][i] + __shfl_xor_sync(0xffffffffu, oacc[dt][i], 2);
+                else
+                    tot[dt][i] = oacc[dt][i] + oacc2[dt][i];
+            }
+        if (writer) {
+            const float inv0 = l2[0] > 0.f ? 1.f / l2[0] : 0.f;
+            const float inv1 = l2[1] > 0.f ? 1.f / l2[1] : 0.f;
+            const bool w0 = gA < a.G, w1 = gA + 1 < a.G;
+            if (r == 0) {
+                if (w0) {
+                    st_cluster_f32(sr.base + 4u * (4 + gA), m2[0]);
+                    st_cluster_f32(sr.base + 4u * (4 + GMAX + gA), l2[0]);
+                }
+                if (w1) {
+                    st_cluster_f32(sr.base + 4u * (4 + gA + 1), m2[1]);
+                    st_cluster_f32(sr.base + 4u * (4 + GMAX + gA + 1), l2[1]);
+                }
+            }
+#pragma unroll
+            for (int dt = 0; dt < KS; ++dt) {
+                const int d = dt * 16 + r;
+                if (w0) {
+                    st_cluster_f32(sr.base + 4u * (u_off + gA * D + d), tot[dt][0] * inv0);
+                    st_cluster_f32(sr.base + 4u * (u_off + gA * D + d + 8), tot[dt][2] * inv0);
+                }
+                if (w1) {
+                    st_cluster_f32(sr.base + 4u * (u_off + (gA + 1) * D + d), tot[dt][1] * inv1);
+                    st_cluster_f32(sr.base + 4u * (u_off + (gA + 1) * D + d + 8), tot[dt][3] * inv1);
+                }
+            }
+        }
+        publish_slot_flag(sr, lane, 0u);
+        mbar_arrive_cluster(sr.ready);
+        return true;
+    }
+};
+
+template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+__device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h, int cw)
+{
+    const int lane = threadIdx.x & 31;
+    using Engine = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX>,
+                                             CudaEngine<T, D, PAGE, GMAX>>::type;
+    Engine eng;
+    eng.load_q(a, b, h, lane);
+    float *pbuf = sh.pbuf + (ENGINE == kEngineMma ? 0 : cw * PAGE * GMAX);
+    const uint32_t ring_cl = mapa(smem_u32(sh.ring), 0);
+    const uint32_t ready_cl = mapa(sh.ready(0, a.S), 0);
+    for (uint32_t i = (uint32_t)cw;; i += (uint32_t)a.NW) {
+        const int s = (int)(i % (uint32_t)a.S);
+        const uint32_t par = (i / (uint32_t)a.S) & 1u;
+        if (!warp_wait<false>(sh.full_k(s), par, sh.abort, a.timeout_ns, a.device_status))
+            break;
+        const uint32_t j = sh.stage_j[s];
+        if (j == kEndOfStream)
+            break;
+        const int nv = (int)sh.stage_nv[s];
+        const uint32_t slot = j % (uint32_t)a.R;
+        SlotRef sr{ring_cl + slot * sh.L.slot_bytes, ready_cl + 8u * slot};
+        if (nv < 0) {  // bad page: forward the flag, free the stage
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(sh.empty(s, a.S));
+            publish_slot_flag(sr, lane, 1u);
+            mbar_arrive_cluster(sr.ready);
+            continue;
+        }
+        if (!eng.block(a, sh, s, par, nv, pbuf, sr, sh.L.u_off_floats, lane))
+            break;
+    }
+}
+
+// ---- merge -----------------------------------------------------------------------
+
+template <int D, int GMAX>
+__device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, int N)
+{
+    constexpr int DE = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int G = a.G;
+    const float eps_m = a.eps_m_arr ? a.eps_m_arr[b] : a.eps_m;
+    const float eps_d = a.eps_d_arr ? a.eps_d_arr[b] : a.eps_d;
+    const int P = a.P_arr ? a.P_arr[b] : a.P;
+    const int minb = a.minb_arr ? a.minb_arr[b] : a.min_blocks;
+    const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
+    const uint32_t u_off = sh.L.u_off_floats;
+
+    float o[GMAX][DE], Mx[GMAX], Lm[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+        Mx[g] = -CUDART_INF_F;
+        Lm[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DE; ++e)
+            o[g][e] = 0.f;
+    }
+    int cnt = 0, stop = 0;
+    bool failed = false;
+    if (a.debug_flags & 1) {
+        // a wait nothing will ever satisfy: exercises the bounded-wait path
+        if (!warp_wait<true>(sh.never(a.S, a.R), 0u, sh.abort, a.timeout_ns, a.device_status))
+            failed = true;
+    }
+    for (int j = 0; !failed && j < N; ++j) {
+        const int slot = j % a.R;
+        if (!warp_wait<true>(sh.ready(slot, a.S), (uint32_t)(j / a.R) & 1u, sh.abort, a.timeout_ns,
+                             a.device_status)) {
+            failed = true;
+            break;
+        }
+        const float *sp = sh.ring + (size_t)slot * (sh.L.slot_bytes / 4);
+        if (__float_as_uint(sp[0]) != 0u) {  // a bad order or page entry upstream
+            failed = true;
+            break;
+        }
+        float n0 = 0.f, Dp = 0.f, Ep = 0.f;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+            if (g < G) {
+                const float mb = sp[4 + g], lb = sp[4 + GMAX + g];
+                float u[DE];
+                if constexpr (DE == 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(sp + u_off + g * D + lane * 4);
+                    u[0] = v.x; u[1] = v.y; u[2] = v.z; u[3] = v.w;
+                } else {
+                    const float2 v = *reinterpret_cast<const float2 *>(sp + u_off + g * D + lane * 2);
+                    u[0] = v.x; u[1] = v.y;
+                }
+                // share of the block in the merged softmax mass (log2 domain)
+                const float Mn = fmaxf(Mx[g], mb);
+                float beta = 0.f;
+                if (Mn != -CUDART_INF_F) {
+                    const float al = exp2f(Mx[g] - Mn);
+                    const float eb = exp2f(mb - Mn);
+                    const float Ln = fmaf(Lm[g], al, lb * eb);
+                    beta = Ln > 0.f ? (lb * eb) / Ln : 0.f;
+                    Mx[g] = Mn;
+                    Lm[g] = Ln;
+                }
+#pragma unroll
+                for (int e = 0; e < DE; ++e) {
+                    const float dl = beta * (u[e] - o[g][e]);
+                    n0 = fmaf(o[g][e], o[g][e], n0);
+                    Dp = fmaf(o[g][e], dl, Dp);
+                    Ep = fmaf(dl, dl, Ep);
+                    o[g][e] += dl;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            st_release_cluster_u32(ctrl_cl, (uint32_t)(j + 1));  // slot consumed
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            n0 += __shfl_xor_sync(0xffffffffu, n0, off);
+            Dp += __shfl_xor_sync(0xffffffffu, Dp, off);
+            Ep += __shfl_xor_sync(0xffffffffu, Ep, off);
+        }
+        if (j >= 1) {
+            // ||o_j||^2 = ||o_{j-1}||^2 + 2 o_{j-1}.Delta + ||Delta||^2; the
+            // direction change uses the part of Delta orthogonal to o_{j-1}.
+            bool stable = false;
+            const float n1sq = n0 + 2.f * Dp + Ep;
+            if (n0 > 0.f && n1sq > 0.f) {
+                const float r0 = sqrtf(n0), r1 = sqrtf(n1sq);
+                const float d_scale = fabsf(2.f * Dp + Ep) / ((r1 + r0) * r0);
+                const float x = r0 + Dp / r0;
+                const float y2 = fmaxf(Ep - (Dp / r0) * (Dp / r0), 0.f);
+                const float d_dir = x > 0.f ? y2 / (r1 * (r1 + x)) : 1.f - x / r1;
+                stable = (d_scale < eps_m) && (d_dir < eps_d);
+            }
+            cnt = stable ? cnt + 1 : 0;
+        }
+        if (cnt >= P && j + 1 >= minb) {
+            stop = j + 1;
+            break;
+        }
+    }
+    if (!failed && stop == 0)
+        stop = N;
+    if (lane == 0)
+        st_release_cluster_u32(ctrl_cl, kStopBit | (uint32_t)(failed ? 0 : stop));
+    float *op = a.out + (int64_t)b * a.out_sb;
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g)
+        if (g < G)
+#pragma unroll
+            for (int e = 0; e < DE; ++e)
+                op[(int64_t)(h * G + g) * a.out_sh + lane * DE + e] = failed ? 0.f : o[g][e];
+    if (lane == 0)
+        a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = failed ? -1 : stop;
+}
+
+// ---- kernel ------------------------------------------------------------------------
+
+template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+    art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    Shared sh;
+    sh.L = make_layout(a.S, a.NW, a.R, PAGE, D, (int)sizeof(T), GMAX, ENGINE != kEngineMma);
+    sh.kv = base + sh.L.kv_off;
+    sh.ring = reinterpret_cast<float *>(base + sh.L.ring_off);
+    sh.pbuf = reinterpret_cast<float *>(base + sh.L.pbuf_off);
+    sh.stage_j = reinterpret_cast<uint32_t *>(base + sh.L.meta_off);
+    sh.stage_nv = sh.stage_j + a.S;
+    sh.bar0 = smem_u32(base + sh.L.bar_off);
+    sh.ctrl = reinterpret_cast<volatile uint32_t *>(base + sh.L.ctrl_off);
+    sh.fetched = sh.ctrl + 1;
+    sh.abort = sh.ctrl + 2;
+
+    const int warp = threadIdx.x >> 5;
+    const uint32_t rank = cluster_ctarank();
+    const int unit = blockIdx.x / a.C;
+    const int b = unit / a.Hkv, h = unit % a.Hkv;
+    const int Lseq = a.seq_lens[b];
+    const int N = Lseq <= 0 ? 0 : (Lseq + PAGE - 1) / PAGE;
+    const bool bad_len = N > a.max_blocks;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.S; ++s) {
+            mbar_init(sh.full_k(s), 1);
+            mbar_init(sh.full_v(s, a.S), 1);
+            mbar_init(sh.empty(s, a.S), 1);
+        }
+        for (int r = 0; r < a.R; ++r)
+            mbar_init(sh.ready(r, a.S), 32);
+        mbar_init(sh.never(a.S, a.R), 1);
+        sh.ctrl[0] = 0u;
+        sh.ctrl[1] = 0u;
+        sh.ctrl[2] = 0u;
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+    cluster_sync();  // remote CTAs may now arrive on the leader's barriers
+
+    if (N > 0 && !bad_len) {
+        if (warp == 0)
+            producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank);
+        else if (warp == 1) {
+            if (rank == 0)
+                merge_role<D, GMAX>(a, sh, b, h, N);
+        } else
+            compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 2);
+    } else if (rank == 0 && warp == 1) {
+        const int lane = threadIdx.x & 31;
+        float *op = a.out + (int64_t)b * a.out_sb;
+        for (int i = lane; i < a.G * D; i += 32)
+            op[(int64_t)(h * a.G + i / D) * a.out_sh + i % D] = 0.f;
+        if (lane == 0) {
+            a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = bad_len ? -1 : 0;
+            if (bad_len)
+                record_error(a.device_status, kErrBadIndex);
+        }
+    }
+    __syncwarp();
+    cluster_sync();  // remote stores into the leader are complete
+    if (rank == 0 && threadIdx.x == 0 && a.blocks_fetched)
+        a.blocks_fetched[unit] = (int32_t)sh.fetched[0];
+}
+
+// Default walk order: [0, N-1, N-2, ..., 1], -1 beyond N.
+__global__ void art_build_order_kernel(const int32_t *seq_lens, int B, int page, int32_t *order, int64_t row_stride,
+                                       int max_blocks)
+{
+    const int b = blockIdx.y;
+    if (b >= B)
+        return;
+    const int L = seq_lens[b];
+    const int N = L <= 0 ? 0 : (L + page - 1) / page;
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < max_blocks; j += gridDim.x * blockDim.x)
+        order[(int64_t)b * row_stride + j] = j < N ? (j == 0 ? 0 : N - j) : -1;
+}
+
+}  // namespace art
