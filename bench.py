@@ -1,0 +1,414 @@
+"""Benchmark: ART decode attention on one B200 (or N independent replicas).
+
+A step is one pass of the whole hot path over one decode batch: the default
+walk order is built on the device (sink block, then newest to oldest), then
+the ART walk runs for every (sequence, kv-head) unit.  The K/V cache is
+resident in HBM before timing starts; the L2 is flushed (a 512 MiB write)
+before every step, outside the step's events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+
+Under torchrun each rank runs its own batch of the same shape (weak scaling,
+no collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ART decode-attn queries/s; KV GB/s read & % of B200 HBM peak; % KV blocks skipped"
+DEFAULT_WORKLOAD = "llama8b_b8"
+WORKLOAD_TEXT = {
+    "tiny_fp32": "tiny fp32: B=1, Hq=Hkv=4, d=64, L=1024, 16-token blocks, 4 planted tokens",
+    "llama8b_b8": "Llama-3-8B-shaped GQA 32/8, d=128, bf16 paged KV, B=8, L=8192, 64-token pages, "
+                  "power-law recency keys",
+    "llama8b_b32": "Llama-3-8B-shaped GQA 32/8, d=128, bf16 paged KV, B=32, L=32768, 64-token pages",
+    "qwen7b_b4": "Qwen2.5-7B-shaped GQA 28/4, d=128, bf16 paged KV, B=4, L=131072, 16 planted heavy hitters",
+    "mistral7b_b128": "Mistral-7B-shaped GQA 32/8, d=128, bf16 paged KV, B=128, ragged L in [1024,16384]",
+}
+SPEC_HBM_GBS = 8000.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
+                "kv_cache_early_art_b200/csrc/art_api.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the walk kernel from the committed ncu summary,
+    only while it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"art_walk_{workload}.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("source_hash") == kernel_source_hash():
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        import tempfile
+        import torch
+        props = torch.cuda.get_device_properties(device)
+        uuid = getattr(props, "uuid", None)
+        self.gpu = f"GPU-{uuid}" if uuid else str(device.index or 0)
+        self.path = tempfile.mktemp(prefix="art_clocks_", suffix=".csv")
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.send_signal(__import__("signal").SIGINT)
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            try:
+                with open(self.path) as f:
+                    self.lines = [l for l in f if l.strip()]
+                os.unlink(self.path)
+            except Exception:
+                self.lines = []
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def replica_seed(rank: int) -> int:
+    """Each replica decodes its own batch: same shape, different draws."""
+    return 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks of a host-side measurement (not a data-path collective)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- oracle ----
+
+def time_oracle(w_cpu, budget_s: float):
+    """The CPU oracle on the whole batch, repeated until budget_s has passed."""
+    import oracle
+    ncores = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.run(w_cpu, want_out=True, nthreads=ncores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return w_cpu.B * reps / el, ncores, reps, el
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    from kv_cache_early_art_b200.workloads import make_workload
+    w = make_workload(args.workload, seed=replica_seed(0), device="cpu")
+    import oracle
+    ncores = os.cpu_count() or 1
+    for _ in range(args.warmup):
+        oracle.run(w, nthreads=ncores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.run(w, nthreads=ncores)
+        times.append(time.perf_counter() - t0)
+    ms = 1000.0 * sum(times) / len(times)
+    value = w.B / (ms / 1000.0)
+    sample = f"whole {args.workload} batch ({w.B} queries, all {w.B * w.Hkv} units) per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_for(args.workload, w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": ncores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_for(name, w, gpus):
+    p = w.uniform_params()
+    cfg = {"workload": f"{name}: {WORKLOAD_TEXT.get(name, name)}", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+           "d": w.d, "page": w.page, "max_seq_len": int(w.seq_lens.max()),
+           "params": ({"eps_m": p[0], "eps_d": p[1], "P": int(p[2]), "min_blocks": int(p[3])} if p else
+                      "per-sequence"),
+           "order": "sink block, then newest to oldest (built on the device each step)",
+           "l2": "flushed before every step (512 MiB write, outside the step events)",
+           "parallelism": f"replicas x{gpus} (independent batches, no collective)"}
+    return cfg
+
+
+# ------------------------------------------------------------------ ours ----
+
+def run_ours(args):
+    import torch
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    import kv_cache_early_art_b200 as art
+    from kv_cache_early_art_b200.workloads import make_workload
+
+    w = make_workload(args.workload, seed=replica_seed(rank), device=dev)
+    B, Hkv, page, d = w.B, w.Hkv, w.page, w.d
+    esize = w.k_cache.element_size()
+    N = w.n_blocks().to(dev)
+    full_blocks = int(N.sum().item()) * Hkv
+    block_bytes = 2 * page * d * esize            # K and V of one page of one kv head
+    uni = w.uniform_params()
+    stream = torch.cuda.current_stream(dev)
+    order = torch.empty_like(w.block_order)
+    fetched = torch.zeros(B * Hkv, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty(B, w.Hq, d, dtype=torch.float32, device=dev)
+    stop = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step(eps_off=False):
+        art.art_build_order_sink_recency(w.seq_lens, page, order)
+        kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
+                  P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
+                  device_status=status, out=out, stop_block=stop)
+        return art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, order, w.seq_lens,
+                                           eps_m=0.0, eps_d=0.0, want_info=True, **kw)
+
+    def timed(n, eps_off=False):
+        """n steps; per step: flush, then [build order | walk] between events.
+        Returns per-step ms and walk-only ms."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for i in range(n):
+            flush.fill_(i)
+            ev[i][0].record(stream)
+            art.art_build_order_sink_recency(w.seq_lens, page, order)
+            ev[i][1].record(stream)
+            kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
+                      P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
+                      device_status=status, out=out, stop_block=stop)
+            art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, order, w.seq_lens,
+                                        eps_m=0.0, eps_d=0.0, **kw)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        return ([e[0].elapsed_time(e[2]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev])
+
+    _, _, info = step()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    # ---- timed region (device time, max over ranks) ----
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clk:
+        step_ms, walk_ms = timed(args.steps)
+    torch.cuda.synchronize(dev)
+    if ws > 1:
+        torch.distributed.barrier()
+    stops = stop.clone()
+    consumed = int(stops.clamp(min=0).sum().item())
+    fetched_blocks = int(fetched.sum().item())
+    assert int(status.item()) == 0
+    ms = sum(step_ms) / len(step_ms)
+    ms_walk = sum(walk_ms) / len(walk_ms)
+    ms_max = reduce_max(ms, ws, dev)
+    queries_all = reduce_sum(float(B), ws, dev)
+    value = queries_all / (ms_max / 1000.0)
+
+    # ---- termination disabled: the same kernel as full attention ----
+    for _ in range(2):
+        step(eps_off=True)
+    f_step, f_walk = timed(max(3, args.steps // 2), eps_off=True)
+    ms_full = sum(f_walk) / len(f_walk)
+    full_consumed = int(stop.clamp(min=0).sum().item())
+
+    alg_bytes = consumed * block_bytes
+    fetch_bytes = fetched_blocks * block_bytes
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / (ms_walk / 1000.0) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": ncu_traffic(args.workload), "peak_kind": peak_kind,
+            "kernel": "art_walk_kernel (walk only; order builder excluded)",
+            "algorithmic_bytes_per_launch": alg_bytes}
+
+    line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": str(w.k_cache.dtype).replace("torch.", "").replace("bfloat16", "bf16"),
+            "data": "synthetic", "config": config_for(args.workload, w, ws),
+            "kv_gbs_fetched": fetch_bytes / (ms_walk / 1000.0) / 1e9,
+            "kv_gbs_algorithmic": achieved,
+            "hbm_frac_of_measured": fetch_bytes / (ms_walk / 1000.0) / 1e9 / peak,
+            "hbm_frac_of_8tbs_spec": fetch_bytes / (ms_walk / 1000.0) / 1e9 / SPEC_HBM_GBS,
+            "skip_frac_blocks": 1.0 - consumed / full_blocks,
+            "fetch_waste_blocks": fetched_blocks - consumed,
+            "walk_ms": ms_walk, "order_ms": ms - ms_walk,
+            "full_attention": {"walk_ms": ms_full, "kv_gbs": full_consumed * block_bytes / (ms_full / 1000.0) / 1e9,
+                               "queries_per_s": B / (ms_full / 1000.0),
+                               "art_speedup": ms_full / ms_walk},
+            "launch": info, "gpu_launches": 2 * args.steps,
+            "roofline": roof, "clocks": clk.summary()}
+
+    # ---- end to end through the public API: pinned host inputs in, results out ----
+    if not args.no_e2e:
+        q_h = w.q.cpu().pin_memory()
+        sl_h = w.seq_lens.cpu().pin_memory()
+        pt_h = w.page_table.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        stop_h = torch.empty(stop.shape, dtype=stop.dtype).pin_memory()
+        q_d, sl_d, pt_d = torch.empty_like(w.q), torch.empty_like(w.seq_lens), torch.empty_like(w.page_table)
+        h2d = q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + pt_h.numel() * 4
+        d2h = out_h.numel() * 4 + stop_h.numel() * 4
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            sl_d.copy_(sl_h, non_blocking=True)
+            pt_d.copy_(pt_h, non_blocking=True)
+            art.art_build_order_sink_recency(sl_d, page, order)
+            art.art_decode_attention_ex(q_d, w.k_cache, w.v_cache, pt_d, order, sl_d, eps_m_per_seq=w.eps_m,
+                                        eps_d_per_seq=w.eps_d, P_per_seq=w.P, min_blocks_per_seq=w.min_blocks,
+                                        out=out, stop_block=stop)
+            out_h.copy_(out, non_blocking=True)
+            stop_h.copy_(stop, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e_ms = []
+        for i in range(args.steps):
+            flush.fill_(i)
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b_.record(stream)
+            b_.synchronize()
+            e_ms.append(a.elapsed_time(b_))
+        em = reduce_max(sum(e_ms) / len(e_ms), ws, dev)
+        line["e2e"] = {"value": queries_all / (em / 1000.0), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": em,
+                       "note": "KV cache resident; per step q, seq_lens, page table in, output and stops out"}
+
+    # ---- CPU oracle baseline (rank 0, N = 1) ----
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        w_cpu = w.to("cpu")
+        qps, cores, reps, el = time_oracle(w_cpu, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                                "sample": f"whole {args.workload} batch ({w.B} queries) x {reps} in {el:.1f} s"}
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -129,8 +129,8 @@ typedef struct {
     int32_t engine;                /* 0 auto, 1 CUDA cores (any dtype), 2 tensor cores (BF16)*/
     int32_t cluster_size;          /* 0 auto, else 1..16 CTAs per unit                      */
     int32_t stages;                /* 0 auto, else 2..8 (a multiple of compute_warps)       */
-    int32_t compute_warps;         /* 0 auto, else 1..8                                     */
-    int32_t window;                /* 0 auto, else 2..64 blocks of speculation              */
+    int32_t compute_warps;         /* 0 auto, else 1..6                                     */
+    int32_t window;                /* 0 auto, else 8..64 blocks of speculation              */
     int64_t timeout_ns;            /* 0 = 2 s; bound on every device-side wait              */
     int32_t debug_flags;           /* 0; bit 0 makes the stop decision wait on a barrier    */
                                    /* nothing arrives on (exercises the bounded wait)       */

@@ -104,10 +104,10 @@ art_status_t check_params(const art_params_t *p)
     if (std::isnan(p->sm_scale) || std::isinf(p->sm_scale))
         return ART_ERR_PARAM;
     if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
-        p->stages > 8 || p->compute_warps < 0 || p->compute_warps > 8 || p->window < 0 || p->window > 64 ||
-        p->timeout_ns < 0 || (p->debug_flags & ~1))
+        p->stages > 8 || p->compute_warps < 0 || p->compute_warps > art::kMaxComputeWarps || p->window < 0 ||
+        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1))
         return ART_ERR_PARAM;
-    if (p->stages == 1 || p->window == 1)
+    if (p->stages == 1 || (p->window > 0 && p->window < art::kMinWindow))
         return ART_ERR_PARAM;
     for (const void *ptr : {(const void *)p->eps_m_per_seq, (const void *)p->eps_d_per_seq,
                             (const void *)p->P_per_seq, (const void *)p->min_blocks_per_seq,
@@ -133,6 +133,22 @@ KernelFn pick_dp(int d, int page)
     if (d == 64)
         return page == 16 ? kfn<T, 64, 16, GMAX, ENGINE>() : kfn<T, 64, 64, GMAX, ENGINE>();
     return page == 16 ? kfn<T, 128, 16, GMAX, ENGINE>() : kfn<T, 128, 64, GMAX, ENGINE>();
+}
+
+template <int ENGINE, int GMAX>
+int merge_warps_dg(int d)
+{
+    return d == 64 ? art::MergeShape<64, GMAX, ENGINE>::NM : art::MergeShape<128, GMAX, ENGINE>::NM;
+}
+
+// warps the kernel instantiation devotes to the merge (compile-time in the kernel)
+int merge_warps(int engine, int d, int gmax)
+{
+    if (engine == art::kEngineMma)
+        return gmax == 4 ? merge_warps_dg<art::kEngineMma, 4>(d) : merge_warps_dg<art::kEngineMma, 8>(d);
+    if (gmax == 1)
+        return merge_warps_dg<art::kEngineCuda, 1>(d);
+    return gmax == 4 ? merge_warps_dg<art::kEngineCuda, 4>(d) : merge_warps_dg<art::kEngineCuda, 8>(d);
 }
 
 int gmax_for(int G, int engine)
@@ -260,15 +276,29 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
     if (s.engine == art::kEngineMma && pr.dtype != ART_BF16)
         return ART_ERR_UNSUPPORTED;
     s.gmax = gmax_for(pr.G, s.engine);
-    s.R = p->window ? p->window : 16;
     s.C = p->cluster_size;
     const int tile = pr.page * pr.d * (int)elem_size(pr.dtype);
-    // (compute warps, stages) in order of preference: about four 16 KiB pages
-    // (or more, smaller ones) in flight, fewer when a large tile must fit
-    static const int small_tiles[][2] = {{4, 8}, {4, 4}, {2, 4}, {2, 2}, {1, 2}};
-    static const int large_tiles[][2] = {{4, 4}, {2, 4}, {2, 2}, {1, 2}};
-    const int(*cand)[2] = tile >= 16384 ? large_tiles : small_tiles;
-    const int ncand = tile >= 16384 ? 4 : 5;
+    const int units = pr.B * pr.Hkv;
+    // (compute warps, stages, window) in order of preference.  With at least
+    // one unit per SM, two small CTAs per SM keep the most pages in flight;
+    // with fewer units each unit is split over a cluster and needs a deeper
+    // window to cover the latency from fetch to merged stop decision.
+    static const int many_units[][3] = {{2, 2, 16}, {1, 2, 16}, {2, 2, 8}, {1, 2, 8}};
+    static const int few_units_large[][3] = {{2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
+    static const int few_units_small[][3] = {{4, 8, 32}, {4, 8, 16}, {4, 4, 16}, {2, 4, 16}, {2, 2, 8},
+                                             {1, 2, 8}};
+    const int(*cand)[3];
+    int ncand;
+    if (units >= di.sms) {
+        cand = many_units;
+        ncand = 4;
+    } else if (tile >= 16384) {
+        cand = few_units_large;
+        ncand = 5;
+    } else {
+        cand = few_units_small;
+        ncand = 6;
+    }
     for (int i = 0; i < ncand; ++i) {
         const int NW = p->compute_warps ? p->compute_warps : cand[i][0];
         int S = p->stages ? p->stages : cand[i][1];
@@ -278,13 +308,14 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
             return ART_ERR_PARAM;
         s.NW = NW;
         s.S = S;
-        s.threads = 32 * (2 + NW);
+        s.R = p->window ? p->window : cand[i][2];
+        s.threads = 32 * (1 + merge_warps(s.engine, pr.d, s.gmax) + NW);
         s.smem = smem_bytes(s, pr);
         if (s.smem <= di.smem_optin) {
             *out = s;
             return ART_OK;
         }
-        if (p->compute_warps && p->stages)
+        if (p->compute_warps && p->stages && p->window)
             break;
     }
     return ART_ERR_UNSUPPORTED;

@@ -39,7 +39,9 @@ namespace art {
 
 constexpr uint32_t kStopBit = 0x80000000u;
 constexpr uint32_t kEndOfStream = 0xFFFFFFFFu;
-constexpr int kMaxThreads = 320;  // producer + merge + up to 8 compute warps
+constexpr int kMaxThreads = 352;  // producer + up to 4 merge + up to 6 compute warps
+constexpr int kMaxComputeWarps = 6;
+constexpr int kMinWindow = 8;     // at least one merge batch
 constexpr int kErrTimeout = -7;
 constexpr int kErrBadIndex = -8;
 constexpr int kEngineCuda = 1;
@@ -74,7 +76,7 @@ struct KernelArgs {
 struct Layout {
     uint32_t tile_bytes, stage_bytes;
     uint32_t kv_off, ring_off, slot_bytes, u_off_floats;
-    uint32_t pbuf_off, meta_off, bar_off, ctrl_off, total;
+    uint32_t pbuf_off, red_off, meta_off, bar_off, ctrl_off, total;
 };
 
 __host__ __device__ inline uint32_t round_up_u32(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -94,6 +96,8 @@ __host__ __device__ inline Layout make_layout(int S, int NW, int R, int page, in
     off += R * L.slot_bytes;
     L.pbuf_off = off;
     off += pbuf ? (uint32_t)(NW * page * gmax * 4) : 0u;
+    L.red_off = off;
+    off += 2 * 4 * 33 * 4;  // merge-warp exchange: 2 batches x up to 4 warps x (32 sums + flag)
     L.meta_off = off;
     off += 2 * S * 4;  // stage_j[S], stage_nv[S]
     off = round_up_u32(off, 8);
@@ -115,8 +119,8 @@ __device__ __forceinline__ void record_error(int32_t *status, int code)
 // trapping) when this CTA was told to abort or when timeout_ns passes; the
 // latter also raises the abort flag and records the timeout.
 template <bool kClusterAcquire>
-__device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int64_t timeout_ns,
-                                       int32_t *status, bool respect_abort = true)
+__device__ __noinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
+                                            int64_t timeout_ns, int32_t *status, bool respect_abort)
 {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
@@ -141,6 +145,16 @@ __device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile u
                 return false;
         }
     }
+}
+
+template <bool kClusterAcquire>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, int64_t timeout_ns,
+                                          int32_t *status, bool respect_abort = true)
+{
+    const bool ok = kClusterAcquire ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, ok))
+        return true;
+    return warp_wait_slow<kClusterAcquire>(bar, parity, abort, timeout_ns, status, respect_abort);
 }
 
 // ---- element loads ---------------------------------------------------------
@@ -211,6 +225,7 @@ struct Shared {
     uint8_t *kv;          // S stages of [K tile | V tile]
     float *ring;          // R slots (meaningful in the leader)
     float *pbuf;          // per compute warp [PAGE][GMAX] (CUDA-core engine)
+    float *red;           // merge-warp exchange
     uint32_t *stage_j, *stage_nv;
     uint32_t bar0;        // shared address of full_k[0]
     volatile uint32_t *ctrl, *fetched, *abort;
@@ -242,6 +257,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
     uint32_t kused = 0, vused = 0;
     uint32_t nfetched = 0;
     int batch_k0 = -1, my_lb = -1, my_pp = -1;
+    uint32_t ctrl_cache = 0;
     bool aborted = false;
 
     auto take_stage = [&](uint32_t i) -> bool {  // wait until stage i % S is free
@@ -270,13 +286,16 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         const int pp = __shfl_sync(0xffffffffu, my_pp, k - batch_k0);
         const bool bad = lb < 0 || lb >= N || pp < 0 || pp >= a.num_pages;
 
-        // speculation window: step j only once j < merged + R
+        // speculation window: step j only once j < merged + R.  The merged
+        // count only grows, so a cached value is re-read when it no longer
+        // admits j, and every fourth step to notice a stop early.
         int go = 1;
-        if (lane == 0) {
+        if (lane == 0 && ((uint32_t)j >= ctrl_cache + (uint32_t)R || (k & 3) == 0)) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const uint32_t c = ld_acquire_cluster_u32(ctrl_cl);
+                const uint32_t c = ld_relaxed_cluster_u32(ctrl_cl);
                 if (c & kStopBit) { go = 0; break; }
+                ctrl_cache = c;
                 if ((uint32_t)j < c + (uint32_t)R) break;
                 if ((it & 15u) == 15u) {
                     const uint64_t now = global_timer_ns();
@@ -377,10 +396,12 @@ struct SlotRef {
     uint32_t ready;  // cluster address of its ready barrier
 };
 
-__device__ __forceinline__ void publish_slot_flag(const SlotRef &sr, int lane, uint32_t flag)
+// Bytes one block state occupies in a slot: flag word, m and l per head,
+// and the normalised output u (all GMAX heads for the tensor-core layout,
+// the G real heads for the CUDA-core layout).
+__device__ __forceinline__ uint32_t slot_tx_bytes(int G, int D, int GMAX, int engine)
 {
-    if (lane == 0)
-        st_cluster_f32(sr.base, __uint_as_float(flag));
+    return 4u + 8u * (uint32_t)G + 4u * (uint32_t)D * (uint32_t)(engine == kEngineMma ? GMAX : G);
 }
 
 // CUDA-core engine: lane l owns head-dim elements [l*DE, l*DE+DE).
@@ -488,10 +509,14 @@ struct CudaEngine {
         if (lane == 0)
             mbar_arrive(sh.empty(s, a.S));
 
-        // block state into the leader's slot
+        // block state into the leader's slot, counted on its ready barrier
+        if (lane == 0) {
+            mbar_arrive_expect_tx_cluster(sr.ready, slot_tx_bytes(a.G, D, GMAX, kEngineCuda));
+            st_async_b32(sr.base, 0u, sr.ready);
+        }
         if (lane < GMAX && lane < a.G) {
-            st_cluster_f32(sr.base + 4u * (4 + lane), m);
-            st_cluster_f32(sr.base + 4u * (4 + GMAX + lane), l);
+            st_async_b32(sr.base + 4u * (4 + lane), __float_as_uint(m), sr.ready);
+            st_async_b32(sr.base + 4u * (4 + GMAX + lane), __float_as_uint(l), sr.ready);
         }
 #pragma unroll
         for (int g = 0; g < GMAX; ++g) {
@@ -500,13 +525,12 @@ struct CudaEngine {
                 const float inv = lg > 0.f ? 1.f / lg : 0.f;
                 const uint32_t addr = sr.base + 4u * (u_off + g * D + lane * DE);
                 if constexpr (DE == 4)
-                    st_cluster_v4(addr, acc[g][0] * inv, acc[g][1] * inv, acc[g][2] * inv, acc[g][3] * inv);
+                    st_async_v4(addr, acc[g][0] * inv, acc[g][1] * inv, acc[g][2] * inv, acc[g][3] * inv,
+                                sr.ready);
                 else
-                    st_cluster_v2(addr, acc[g][0] * inv, acc[g][1] * inv);
+                    st_async_v2(addr, acc[g][0] * inv, acc[g][1] * inv, sr.ready);
             }
         }
-        publish_slot_flag(sr, lane, 0u);
-        mbar_arrive_cluster(sr.ready);
         return true;
     }
 };
@@ -659,35 +683,33 @@ struct MmaEngine {
                 else
                     tot[dt][i] = oacc[dt][i] + oacc2[dt][i];
             }
+        // slot layout of this engine: 16-byte vectors, vector (dt, r, c) holds
+        // u[gA][d], u[gA+1][d], u[gA][d+8], u[gA+1][d+8] with d = 16 dt + r
+        if (lane == 0) {
+            mbar_arrive_expect_tx_cluster(sr.ready, slot_tx_bytes(a.G, D, GMAX, kEngineMma));
+            st_async_b32(sr.base, 0u, sr.ready);
+        }
         if (writer) {
-            const float inv0 = l2[0] > 0.f ? 1.f / l2[0] : 0.f;
-            const float inv1 = l2[1] > 0.f ? 1.f / l2[1] : 0.f;
             const bool w0 = gA < a.G, w1 = gA + 1 < a.G;
+            const float inv0 = (w0 && l2[0] > 0.f) ? 1.f / l2[0] : 0.f;
+            const float inv1 = (w1 && l2[1] > 0.f) ? 1.f / l2[1] : 0.f;
             if (r == 0) {
                 if (w0) {
-                    st_cluster_f32(sr.base + 4u * (4 + gA), m2[0]);
-                    st_cluster_f32(sr.base + 4u * (4 + GMAX + gA), l2[0]);
+                    st_async_b32(sr.base + 4u * (4 + gA), __float_as_uint(m2[0]), sr.ready);
+                    st_async_b32(sr.base + 4u * (4 + GMAX + gA), __float_as_uint(l2[0]), sr.ready);
                 }
                 if (w1) {
-                    st_cluster_f32(sr.base + 4u * (4 + gA + 1), m2[1]);
-                    st_cluster_f32(sr.base + 4u * (4 + GMAX + gA + 1), l2[1]);
+                    st_async_b32(sr.base + 4u * (4 + gA + 1), __float_as_uint(m2[1]), sr.ready);
+                    st_async_b32(sr.base + 4u * (4 + GMAX + gA + 1), __float_as_uint(l2[1]), sr.ready);
                 }
             }
+            constexpr int WPT = kShared ? 16 : 32;  // writer lanes per head-dim tile
+            const int widx = kShared ? (r * 2 + c) : (r * 4 + c);
 #pragma unroll
-            for (int dt = 0; dt < KS; ++dt) {
-                const int d = dt * 16 + r;
-                if (w0) {
-                    st_cluster_f32(sr.base + 4u * (u_off + gA * D + d), tot[dt][0] * inv0);
-                    st_cluster_f32(sr.base + 4u * (u_off + gA * D + d + 8), tot[dt][2] * inv0);
-                }
-                if (w1) {
-                    st_cluster_f32(sr.base + 4u * (u_off + (gA + 1) * D + d), tot[dt][1] * inv1);
-                    st_cluster_f32(sr.base + 4u * (u_off + (gA + 1) * D + d + 8), tot[dt][3] * inv1);
-                }
-            }
+            for (int dt = 0; dt < KS; ++dt)
+                st_async_v4(sr.base + 4u * (u_off + 4 * (dt * WPT + widx)), tot[dt][0] * inv0, tot[dt][1] * inv1,
+                            tot[dt][2] * inv0, tot[dt][3] * inv1, sr.ready);
         }
-        publish_slot_flag(sr, lane, 0u);
-        mbar_arrive_cluster(sr.ready);
         return true;
     }
 };
@@ -718,8 +740,10 @@ __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(sh.empty(s, a.S));
-            publish_slot_flag(sr, lane, 1u);
-            mbar_arrive_cluster(sr.ready);
+            if (lane == 0) {
+                mbar_arrive_expect_tx_cluster(sr.ready, 4u);
+                st_async_b32(sr.base, 1u, sr.ready);
+            }
             continue;
         }
         if (!eng.block(a, sh, s, par, nv, pbuf, sr, sh.L.u_off_floats, lane))
@@ -729,10 +753,65 @@ __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h
 
 // ---- merge -----------------------------------------------------------------------
 
+// Which slot floats a merge lane owns.  The lane keeps the running output for
+// NV vectors of VW floats; element e of vector i belongs to head
+// head(lane, i, e) and head-dim index dim(lane, i, e).
+template <int D, int GMAX, int ENGINE>
+struct MergeLayout {  // CUDA-core slots: u[g][d]; lane owns d in [lane*DE, lane*DE+DE) of every head
+    static constexpr int VW = D / 32, NV = GMAX;
+    static constexpr bool kTwoHeads = false;
+    __device__ static int off(int lane, int i) { return i * D + lane * VW; }
+    __device__ static int head(int, int i, int) { return i; }
+    __device__ static int dim(int lane, int, int e) { return lane * VW + e; }
+};
 template <int D, int GMAX>
-__device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, int N)
+struct MergeLayout<D, GMAX, kEngineMma> {  // tensor-core slots: vector v = dt*W + r*C + c
+    static constexpr int W = GMAX <= 4 ? 16 : 32, CW = GMAX <= 4 ? 2 : 4;
+    static constexpr int VW = 4, NV = (D / 16) * W / 32;
+    static constexpr bool kTwoHeads = true;
+    __device__ static int off(int lane, int i) { return 4 * (lane + 32 * i); }
+    __device__ static int head(int lane, int, int e) { return 2 * (lane % CW) + (e & 1); }
+    __device__ static int dim(int lane, int i, int e)
+    {
+        const int v = lane + 32 * i;
+        return (v / W) * 16 + (v % W) / CW + (e >> 1) * 8;
+    }
+};
+
+// How the merge is split: NM warps share the output elements (vectors
+// [mw*NVW, mw*NVW+NVW) of every lane belong to merge warp mw); KB blocks are
+// folded per batch, with one scan lane per (block, head) pair.
+template <int D, int GMAX, int ENGINE>
+struct MergeShape {
+    using Lay = MergeLayout<D, GMAX, ENGINE>;
+    static constexpr int TOT = Lay::NV * Lay::VW;
+    static constexpr int NM = TOT / 16 < 1 ? 1 : (TOT / 16 > 4 ? 4 : TOT / 16);
+    static constexpr int NVW = Lay::NV / NM;
+    static constexpr int KB = (32 / GMAX) < 8 ? (32 / GMAX) : 8;
+    static_assert(Lay::NV % NM == 0, "merge split");
+};
+
+__device__ __forceinline__ void merge_barrier(int nthreads)
 {
-    constexpr int DE = D / 32;
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Folds block states into the running output in walk order, KB blocks per
+// batch.  Per batch: wait for the KB states; one lane per (block, head) forms
+// the blocks' shares of the softmax mass with a prefix scan (block max, then
+// prefix sums of l 2^(m - M)); every merge warp folds the blocks into its
+// slice of o, accumulating ||o_{j-1}||^2, o_{j-1}.Delta_j and ||Delta_j||^2;
+// the slices' sums meet in shared memory; every merge warp then evaluates the
+// statistics of the batch's blocks lane-parallel and runs the patience rule,
+// reaching the same decision.  A stop inside a batch replays the batch up to
+// the stop from a snapshot, so the stop and the output are those of a
+// strictly sequential walk.
+template <int D, int GMAX, int ENGINE>
+__device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, int N, int mw)
+{
+    using MS = MergeShape<D, GMAX, ENGINE>;
+    using Lay = typename MS::Lay;
+    constexpr int NVW = MS::NVW, VW = Lay::VW, KB = MS::KB, NM = MS::NM;
     const int lane = threadIdx.x & 31;
     const int G = a.G;
     const float eps_m = a.eps_m_arr ? a.eps_m_arr[b] : a.eps_m;
@@ -741,16 +820,20 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     const int minb = a.minb_arr ? a.minb_arr[b] : a.min_blocks;
     const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
     const uint32_t u_off = sh.L.u_off_floats;
+    const int slot_floats = (int)(sh.L.slot_bytes / 4);
+    const int vbase = mw * NVW;
 
-    float o[GMAX][DE], Mx[GMAX], Lm[GMAX];
+    // scan lane: block kl of the batch, head gl; it also keeps the running
+    // softmax scalars of head gl
+    const int kl = lane / GMAX, gl = lane % GMAX;
+    float Mx = -CUDART_INF_F, Lm = 0.f;
+    float o[NVW][VW];
 #pragma unroll
-    for (int g = 0; g < GMAX; ++g) {
-        Mx[g] = -CUDART_INF_F;
-        Lm[g] = 0.f;
+    for (int i = 0; i < NVW; ++i)
 #pragma unroll
-        for (int e = 0; e < DE; ++e)
-            o[g][e] = 0.f;
-    }
+        for (int e = 0; e < VW; ++e)
+            o[i][e] = 0.f;
+
     int cnt = 0, stop = 0;
     bool failed = false;
     if (a.debug_flags & 1) {
@@ -758,93 +841,238 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         if (!warp_wait<true>(sh.never(a.S, a.R), 0u, sh.abort, a.timeout_ns, a.device_status))
             failed = true;
     }
-    for (int j = 0; !failed && j < N; ++j) {
-        const int slot = j % a.R;
-        if (!warp_wait<true>(sh.ready(slot, a.S), (uint32_t)(j / a.R) & 1u, sh.abort, a.timeout_ns,
-                             a.device_status)) {
-            failed = true;
-            break;
-        }
-        const float *sp = sh.ring + (size_t)slot * (sh.L.slot_bytes / 4);
-        if (__float_as_uint(sp[0]) != 0u) {  // a bad order or page entry upstream
-            failed = true;
-            break;
-        }
-        float n0 = 0.f, Dp = 0.f, Ep = 0.f;
+
+    // fold batch block k (slot pointer sp) into this warp's slice of o, given
+    // this lane's u vectors uv; partial sums into pn, pd, pe
+    auto fold = [&](int k, float beta, const float (&uv)[NVW][VW], float &pn, float &pd, float &pe) {
+        float bsel[Lay::kTwoHeads ? 2 : NVW];
+        if constexpr (Lay::kTwoHeads) {
+            const int h0 = Lay::head(lane, 0, 0);
+            bsel[0] = __shfl_sync(0xffffffffu, beta, k * GMAX + h0);
+            bsel[1] = __shfl_sync(0xffffffffu, beta, k * GMAX + h0 + 1);
+        } else {
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) {
-            if (g < G) {
-                const float mb = sp[4 + g], lb = sp[4 + GMAX + g];
-                float u[DE];
-                if constexpr (DE == 4) {
-                    const float4 v = *reinterpret_cast<const float4 *>(sp + u_off + g * D + lane * 4);
-                    u[0] = v.x; u[1] = v.y; u[2] = v.z; u[3] = v.w;
-                } else {
-                    const float2 v = *reinterpret_cast<const float2 *>(sp + u_off + g * D + lane * 2);
-                    u[0] = v.x; u[1] = v.y;
-                }
-                // share of the block in the merged softmax mass (log2 domain)
-                const float Mn = fmaxf(Mx[g], mb);
-                float beta = 0.f;
-                if (Mn != -CUDART_INF_F) {
-                    const float al = exp2f(Mx[g] - Mn);
-                    const float eb = exp2f(mb - Mn);
-                    const float Ln = fmaf(Lm[g], al, lb * eb);
-                    beta = Ln > 0.f ? (lb * eb) / Ln : 0.f;
-                    Mx[g] = Mn;
-                    Lm[g] = Ln;
-                }
+            for (int ii = 0; ii < NVW; ++ii)
+                bsel[ii] = __shfl_sync(0xffffffffu, beta, k * GMAX + vbase + ii);
+        }
 #pragma unroll
-                for (int e = 0; e < DE; ++e) {
-                    const float dl = beta * (u[e] - o[g][e]);
-                    n0 = fmaf(o[g][e], o[g][e], n0);
-                    Dp = fmaf(o[g][e], dl, Dp);
-                    Ep = fmaf(dl, dl, Ep);
-                    o[g][e] += dl;
+        for (int ii = 0; ii < NVW; ++ii) {
+            if (!Lay::kTwoHeads && vbase + ii >= G)
+                continue;
+#pragma unroll
+            for (int e = 0; e < VW; ++e) {
+                const float bt = Lay::kTwoHeads ? bsel[e & 1] : bsel[Lay::kTwoHeads ? 0 : ii];
+                const float dl = bt * (uv[ii][e] - o[ii][e]);
+                pn = fmaf(o[ii][e], o[ii][e], pn);
+                pd = fmaf(o[ii][e], dl, pd);
+                pe = fmaf(dl, dl, pe);
+                o[ii][e] += dl;
+            }
+        }
+    };
+    auto load_u = [&](const float *sp, float (&uv)[NVW][VW]) {
+#pragma unroll
+        for (int ii = 0; ii < NVW; ++ii) {
+            const float *up = sp + u_off + Lay::off(lane, vbase + ii);
+            if constexpr (VW == 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(up);
+                uv[ii][0] = x.x; uv[ii][1] = x.y; uv[ii][2] = x.z; uv[ii][3] = x.w;
+            } else {
+                const float2 x = *reinterpret_cast<const float2 *>(up);
+                uv[ii][0] = x.x; uv[ii][1] = x.y;
+            }
+        }
+    };
+    // fold blocks 0..kend of the batch starting at slot s0 (u loads one block ahead)
+    auto fold_batch = [&](int s0, int kend, float beta, float (&v)[32], bool sums) {
+        float ua[NVW][VW], ub[NVW][VW];
+        load_u(sh.ring + (size_t)s0 * slot_floats, ua);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            if (k > kend)
+                break;
+            if (k + 1 <= kend) {
+                int sn = s0 + k + 1;
+                sn = sn >= a.R ? sn - a.R : sn;
+                load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
+            }
+            float t0 = 0.f, t1 = 0.f, t2 = 0.f;
+            fold(k, beta, (k & 1) ? ub : ua, sums ? v[4 * k] : t0, sums ? v[4 * k + 1] : t1, sums ? v[4 * k + 2] : t2);
+        }
+    };
+
+    int s0 = 0;        // slot of the batch's first block, j0 % R
+    uint32_t ph0 = 0;  // parity of that slot's phase, (j0 / R) & 1
+    for (int j0 = 0, batch = 0; !failed && stop == 0 && j0 < N; j0 += KB, ++batch) {
+        const int nb = min(KB, N - j0);
+        // 1. the batch's block states: lane k polls block j0 + k; a flagged
+        //    state (bad order or page entry upstream) ends the walk
+        int sk = s0 + (lane < KB ? lane : 0);
+        uint32_t pk = ph0;
+        if (sk >= a.R) {
+            sk -= a.R;
+            pk ^= 1u;
+        }
+        const float *spk = sh.ring + (size_t)sk * slot_floats;
+        bool local_fail = false;
+        {
+            uint64_t t0 = 0;
+            for (uint32_t it = 0;; ++it) {
+                const bool arrived = lane >= nb || mbar_try_wait(sh.ready(sk, a.S), pk);
+                if (__any_sync(0xffffffffu, arrived && lane < nb && __float_as_uint(spk[0]) != 0u)) {
+                    local_fail = true;
+                    break;
+                }
+                if (__all_sync(0xffffffffu, arrived))
+                    break;
+                if ((it & 7u) == 7u) {
+                    int quit = 0;
+                    if (lane == 0) {
+                        const uint64_t now = global_timer_ns();
+                        if (t0 == 0)
+                            t0 = now;
+                        if (*sh.abort) {
+                            quit = 1;
+                        } else if ((int64_t)(now - t0) > a.timeout_ns) {
+                            *sh.abort = 1u;
+                            record_error(a.device_status, kErrTimeout);
+                            quit = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, quit, 0)) {
+                        local_fail = true;
+                        break;
+                    }
                 }
             }
         }
-        __syncwarp();
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            v[q] = 0.f;
+        float beta = 0.f;
+        float o0[NVW][VW];
+        if (!local_fail) {
+            // 2. shares of the softmax mass: beta_(k,g) = w_k / (L_prev + w_0 + ... + w_k)
+            float mk = -CUDART_INF_F, lk = 0.f;
+            if (kl < nb && gl < G) {
+                int sl = s0 + kl;
+                sl = sl >= a.R ? sl - a.R : sl;
+                const float *sp = sh.ring + (size_t)sl * slot_floats;
+                mk = sp[4 + gl];
+                lk = sp[4 + GMAX + gl];
+            }
+            float Mb = fmaxf(Mx, mk);
+#pragma unroll
+            for (int off = GMAX; off < 32; off <<= 1)
+                Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
+            const float w = (mk == -CUDART_INF_F) ? 0.f : lk * ex2_approx(mk - Mb);
+            float S = w;
+#pragma unroll
+            for (int off = GMAX; off < 32; off <<= 1) {
+                const float t = __shfl_up_sync(0xffffffffu, S, off);
+                if (lane >= off)
+                    S += t;
+            }
+            const float Lam = ((Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb)) + S;
+            beta = Lam > 0.f ? w * rcp_approx(Lam) : 0.f;
+            Lm = __shfl_sync(0xffffffffu, Lam, (nb - 1) * GMAX + gl);
+            Mx = Mb;
+            // 3. fold the batch into this warp's slice
+#pragma unroll
+            for (int i = 0; i < NVW; ++i)
+#pragma unroll
+                for (int e = 0; e < VW; ++e)
+                    o0[i][e] = o[i][e];
+            fold_batch(s0, nb - 1, beta, v, true);
+            reduce_scatter32(v, lane);  // lane 4k+q: quantity q of batch block k
+        }
+        // 4. the slices meet; a failure anywhere ends the walk for every merge warp
+        float *red = sh.red + (batch & 1) * (NM * 33);
+        red[mw * 33 + lane] = v[0];
         if (lane == 0)
-            st_release_cluster_u32(ctrl_cl, (uint32_t)(j + 1));  // slot consumed
+            reinterpret_cast<volatile int *>(red)[mw * 33 + 32] = local_fail ? 1 : 0;
+        if constexpr (NM > 1)
+            merge_barrier(NM * 32);
+        else
+            __syncwarp();
+        bool any_fail = false;
+        float tot = 0.f;
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            n0 += __shfl_xor_sync(0xffffffffu, n0, off);
-            Dp += __shfl_xor_sync(0xffffffffu, Dp, off);
-            Ep += __shfl_xor_sync(0xffffffffu, Ep, off);
+        for (int w2 = 0; w2 < NM; ++w2) {
+            any_fail |= reinterpret_cast<volatile int *>(red)[w2 * 33 + 32] != 0;
+            tot += red[w2 * 33 + lane];
         }
-        if (j >= 1) {
-            // ||o_j||^2 = ||o_{j-1}||^2 + 2 o_{j-1}.Delta + ||Delta||^2; the
-            // direction change uses the part of Delta orthogonal to o_{j-1}.
-            bool stable = false;
-            const float n1sq = n0 + 2.f * Dp + Ep;
-            if (n0 > 0.f && n1sq > 0.f) {
-                const float r0 = sqrtf(n0), r1 = sqrtf(n1sq);
-                const float d_scale = fabsf(2.f * Dp + Ep) / ((r1 + r0) * r0);
-                const float x = r0 + Dp / r0;
-                const float y2 = fmaxf(Ep - (Dp / r0) * (Dp / r0), 0.f);
-                const float d_dir = x > 0.f ? y2 / (r1 * (r1 + x)) : 1.f - x / r1;
-                stable = (d_scale < eps_m) && (d_dir < eps_d);
-            }
-            cnt = stable ? cnt + 1 : 0;
-        }
-        if (cnt >= P && j + 1 >= minb) {
-            stop = j + 1;
+        if (any_fail) {
+            failed = true;
             break;
+        }
+        // 5. statistics of batch block k in lane 4k, then patience in walk order.
+        // ||o_j||^2 = ||o_{j-1}||^2 + 2 o_{j-1}.Delta + ||Delta||^2; the direction
+        // change uses the part of Delta orthogonal to o_{j-1}.
+        const int base = lane & ~3;
+        const float n0 = __shfl_sync(0xffffffffu, tot, base);
+        const float Dp = __shfl_sync(0xffffffffu, tot, base + 1);
+        const float Ep = __shfl_sync(0xffffffffu, tot, base + 2);
+        bool stable = false;
+        const float n1sq = n0 + 2.f * Dp + Ep;
+        if (n0 > 0.f && n1sq > 0.f) {
+            const float r0 = sqrtf(n0), r1 = sqrtf(n1sq);
+            const float d_scale = fabsf(2.f * Dp + Ep) / ((r1 + r0) * r0);
+            const float x = r0 + Dp / r0;
+            const float y2 = fmaxf(Ep - (Dp / r0) * (Dp / r0), 0.f);
+            const float d_dir = x > 0.f ? y2 / (r1 * (r1 + x)) : 1.f - x / r1;
+            stable = (d_scale < eps_m) && (d_dir < eps_d);
+        }
+        const uint32_t smask = __ballot_sync(0xffffffffu, stable && (lane & 3) == 0);
+        int kstop = -1;
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            const int j = j0 + k;
+            if (kstop < 0 && k < nb) {
+                if (j >= 1)
+                    cnt = (smask >> (4 * k) & 1u) ? cnt + 1 : 0;
+                if (cnt >= P && j + 1 >= minb)
+                    kstop = k;
+            }
+        }
+        if (kstop >= 0) {
+            stop = j0 + kstop + 1;
+            if (kstop < nb - 1) {  // replay the batch up to the stop block
+#pragma unroll
+                for (int i = 0; i < NVW; ++i)
+#pragma unroll
+                    for (int e = 0; e < VW; ++e)
+                        o[i][e] = o0[i][e];
+                fold_batch(s0, kstop, beta, v, false);
+            }
+        }
+        // Slots of this batch are free again (or the walk is over).  Every value
+        // read from them has already fed the decision above, so a relaxed store
+        // cannot overtake those reads.
+        if (mw == 0 && lane == 0)
+            st_relaxed_cluster_u32(ctrl_cl, stop ? (kStopBit | (uint32_t)stop) : (uint32_t)(j0 + nb));
+        s0 += KB;
+        if (s0 >= a.R) {
+            s0 -= a.R;
+            ph0 ^= 1u;
         }
     }
     if (!failed && stop == 0)
         stop = N;
-    if (lane == 0)
-        st_release_cluster_u32(ctrl_cl, kStopBit | (uint32_t)(failed ? 0 : stop));
+    if (failed && mw == 0 && lane == 0)
+        st_relaxed_cluster_u32(ctrl_cl, kStopBit);
     float *op = a.out + (int64_t)b * a.out_sb;
 #pragma unroll
-    for (int g = 0; g < GMAX; ++g)
-        if (g < G)
+    for (int ii = 0; ii < NVW; ++ii)
 #pragma unroll
-            for (int e = 0; e < DE; ++e)
-                op[(int64_t)(h * G + g) * a.out_sh + lane * DE + e] = failed ? 0.f : o[g][e];
-    if (lane == 0)
+        for (int e = 0; e < VW; ++e) {
+            const int i = vbase + ii;
+            const int g = Lay::head(lane, i, e);
+            if (g < G && (Lay::kTwoHeads || i < G))
+                op[(int64_t)(h * G + g) * a.out_sh + Lay::dim(lane, i, e)] = failed ? 0.f : o[ii][e];
+        }
+    if (mw == 0 && lane == 0)
         a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = failed ? -1 : stop;
 }
 
@@ -863,6 +1091,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     sh.kv = base + sh.L.kv_off;
     sh.ring = reinterpret_cast<float *>(base + sh.L.ring_off);
     sh.pbuf = reinterpret_cast<float *>(base + sh.L.pbuf_off);
+    sh.red = reinterpret_cast<float *>(base + sh.L.red_off);
     sh.stage_j = reinterpret_cast<uint32_t *>(base + sh.L.meta_off);
     sh.stage_nv = sh.stage_j + a.S;
     sh.bar0 = smem_u32(base + sh.L.bar_off);
@@ -885,7 +1114,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             mbar_init(sh.empty(s, a.S), 1);
         }
         for (int r = 0; r < a.R; ++r)
-            mbar_init(sh.ready(r, a.S), 32);
+            mbar_init(sh.ready(r, a.S), 1);
         mbar_init(sh.never(a.S, a.R), 1);
         sh.ctrl[0] = 0u;
         sh.ctrl[1] = 0u;
@@ -895,14 +1124,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     __syncthreads();
     cluster_sync();  // remote CTAs may now arrive on the leader's barriers
 
+    constexpr int NM = MergeShape<D, GMAX, ENGINE>::NM;
     if (N > 0 && !bad_len) {
         if (warp == 0)
             producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank);
-        else if (warp == 1) {
+        else if (warp <= NM) {
             if (rank == 0)
-                merge_role<D, GMAX>(a, sh, b, h, N);
+                merge_role<D, GMAX, ENGINE>(a, sh, b, h, N, warp - 1);
         } else
-            compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 2);
+            compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM);
     } else if (rank == 0 && warp == 1) {
         const int lane = threadIdx.x & 31;
         float *op = a.out + (int64_t)b * a.out_sb;
