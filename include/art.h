@@ -110,8 +110,9 @@ typedef struct {
     int32_t threads;       /* threads per CTA                                             */
     int32_t stages;        /* K/V pages buffered per CTA                                  */
     int32_t compute_warps; /* warps turning pages into block states, per CTA              */
-    int32_t window;        /* blocks the walk may fetch ahead of the stop decision        */
+    int32_t window;        /* blocks staged ahead of the merged prefix (state ring slots)  */
     int32_t smem_bytes;    /* dynamic shared memory per CTA                               */
+    int32_t prefetch;      /* further blocks pulled into L2 ahead of the staged ones      */
 } art_launch_info_t;
 
 typedef struct {
@@ -135,6 +136,9 @@ typedef struct {
     int32_t debug_flags;           /* 0; bit 0 makes the stop decision wait on a barrier    */
                                    /* nothing arrives on (exercises the bounded wait)       */
     art_launch_info_t *info;       /* host pointer or NULL                                  */
+    int32_t prefetch;              /* 0 or -1 off, else 1..64 blocks pulled into L2         */
+                                   /* ahead of the staged loads.  Pages read past the stop  */
+                                   /* stay below window + prefetch blocks.                  */
 } art_params_t;
 
 /*

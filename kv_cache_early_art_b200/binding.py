@@ -40,7 +40,7 @@ class ArtTensor(ctypes.Structure):
 
 class ArtLaunchInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("engine", "cluster_size", "grid", "threads", "stages",
-                                               "compute_warps", "window", "smem_bytes")]
+                                               "compute_warps", "window", "smem_bytes", "prefetch")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -56,7 +56,7 @@ class ArtParams(ctypes.Structure):
         ("blocks_fetched", ctypes.c_void_p), ("device_status", ctypes.c_void_p),
         ("engine", ctypes.c_int32), ("cluster_size", ctypes.c_int32), ("stages", ctypes.c_int32),
         ("compute_warps", ctypes.c_int32), ("window", ctypes.c_int32), ("timeout_ns", ctypes.c_int64),
-        ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo))]
+        ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo)), ("prefetch", ctypes.c_int32)]
 
 
 _P = ctypes.POINTER
@@ -138,7 +138,7 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
                             P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                             P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                             engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                            debug_flags=0, out=None, stop_block=None, stream=None, want_info=False):
+                            debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None, want_info=False):
     """art_decode_attention_ex in art.h.  Per-sequence arrays are device
     tensors of length B (float32 thresholds, int32 P / min_blocks).
     Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
@@ -167,6 +167,7 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p.engine, p.cluster_size, p.stages = int(engine), int(cluster_size), int(stages)
     p.compute_warps, p.window, p.timeout_ns = int(compute_warps), int(window), int(timeout_ns)
     p.debug_flags = int(debug_flags)
+    p.prefetch = int(prefetch)
     info = ArtLaunchInfo()
     p.info = ctypes.pointer(info)
     st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))

@@ -105,7 +105,7 @@ art_status_t check_params(const art_params_t *p)
         return ART_ERR_PARAM;
     if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
         p->stages > 8 || p->compute_warps < 0 || p->compute_warps > art::kMaxComputeWarps || p->window < 0 ||
-        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1))
+        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64)
         return ART_ERR_PARAM;
     if (p->stages == 1 || (p->window > 0 && p->window < art::kMinWindow))
         return ART_ERR_PARAM;
@@ -121,34 +121,40 @@ art_status_t check_params(const art_params_t *p)
 
 using KernelFn = void (*)(KernelArgs, CUtensorMap, CUtensorMap);
 
-template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW>
 KernelFn kfn()
 {
-    return art::art_walk_kernel<T, D, PAGE, GMAX, ENGINE>;
+    return art::art_walk_kernel<T, D, PAGE, GMAX, ENGINE, NMW>;
 }
 
-template <typename T, int ENGINE, int GMAX>
+template <typename T, int ENGINE, int GMAX, int NMW>
 KernelFn pick_dp(int d, int page)
 {
     if (d == 64)
-        return page == 16 ? kfn<T, 64, 16, GMAX, ENGINE>() : kfn<T, 64, 64, GMAX, ENGINE>();
-    return page == 16 ? kfn<T, 128, 16, GMAX, ENGINE>() : kfn<T, 128, 64, GMAX, ENGINE>();
+        return page == 16 ? kfn<T, 64, 16, GMAX, ENGINE, NMW>() : kfn<T, 64, 64, GMAX, ENGINE, NMW>();
+    return page == 16 ? kfn<T, 128, 16, GMAX, ENGINE, NMW>() : kfn<T, 128, 64, GMAX, ENGINE, NMW>();
 }
 
-template <int ENGINE, int GMAX>
+template <int ENGINE, int GMAX, int NMW>
 int merge_warps_dg(int d)
 {
-    return d == 64 ? art::MergeShape<64, GMAX, ENGINE>::NM : art::MergeShape<128, GMAX, ENGINE>::NM;
+    return d == 64 ? art::MergeShape<64, GMAX, ENGINE, NMW>::NM : art::MergeShape<128, GMAX, ENGINE, NMW>::NM;
 }
 
-// warps the kernel instantiation devotes to the merge (compile-time in the kernel)
-int merge_warps(int engine, int d, int gmax)
+// Warps the kernel instantiation devotes to the merge (compile-time in the
+// kernel).  Four merge warps shorten the per-unit merge when units are few;
+// one keeps CTAs small enough for two per SM when units are many.  The
+// CUDA-core engine always uses one.
+int merge_warps(int engine, int d, int gmax, int nmw)
 {
-    if (engine == art::kEngineMma)
-        return gmax == 4 ? merge_warps_dg<art::kEngineMma, 4>(d) : merge_warps_dg<art::kEngineMma, 8>(d);
+    if (engine == art::kEngineMma) {
+        if (nmw == 4)
+            return gmax == 4 ? merge_warps_dg<art::kEngineMma, 4, 4>(d) : merge_warps_dg<art::kEngineMma, 8, 4>(d);
+        return gmax == 4 ? merge_warps_dg<art::kEngineMma, 4, 1>(d) : merge_warps_dg<art::kEngineMma, 8, 1>(d);
+    }
     if (gmax == 1)
-        return merge_warps_dg<art::kEngineCuda, 1>(d);
-    return gmax == 4 ? merge_warps_dg<art::kEngineCuda, 4>(d) : merge_warps_dg<art::kEngineCuda, 8>(d);
+        return merge_warps_dg<art::kEngineCuda, 1, 1>(d);
+    return gmax == 4 ? merge_warps_dg<art::kEngineCuda, 4, 1>(d) : merge_warps_dg<art::kEngineCuda, 8, 1>(d);
 }
 
 int gmax_for(int G, int engine)
@@ -158,20 +164,23 @@ int gmax_for(int G, int engine)
     return G <= 1 ? 1 : (G <= 4 ? 4 : 8);
 }
 
-KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax)
+KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax, int nmw)
 {
     if (dtype == ART_F32) {
-        if (gmax == 1) return pick_dp<float, art::kEngineCuda, 1>(d, page);
-        if (gmax == 4) return pick_dp<float, art::kEngineCuda, 4>(d, page);
-        return pick_dp<float, art::kEngineCuda, 8>(d, page);
+        if (gmax == 1) return pick_dp<float, art::kEngineCuda, 1, 1>(d, page);
+        if (gmax == 4) return pick_dp<float, art::kEngineCuda, 4, 1>(d, page);
+        return pick_dp<float, art::kEngineCuda, 8, 1>(d, page);
     }
     if (engine == art::kEngineMma) {
-        if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineMma, 4>(d, page);
-        return pick_dp<__nv_bfloat16, art::kEngineMma, 8>(d, page);
+        if (nmw == 4)
+            return gmax == 4 ? pick_dp<__nv_bfloat16, art::kEngineMma, 4, 4>(d, page)
+                             : pick_dp<__nv_bfloat16, art::kEngineMma, 8, 4>(d, page);
+        return gmax == 4 ? pick_dp<__nv_bfloat16, art::kEngineMma, 4, 1>(d, page)
+                         : pick_dp<__nv_bfloat16, art::kEngineMma, 8, 1>(d, page);
     }
-    if (gmax == 1) return pick_dp<__nv_bfloat16, art::kEngineCuda, 1>(d, page);
-    if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineCuda, 4>(d, page);
-    return pick_dp<__nv_bfloat16, art::kEngineCuda, 8>(d, page);
+    if (gmax == 1) return pick_dp<__nv_bfloat16, art::kEngineCuda, 1, 1>(d, page);
+    if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineCuda, 4, 1>(d, page);
+    return pick_dp<__nv_bfloat16, art::kEngineCuda, 8, 1>(d, page);
 }
 
 // ------------------------------------------------------ device caches ----
@@ -259,7 +268,7 @@ art_status_t make_cache_map(CUtensorMap *map, const art_tensor_t *c, int dtype, 
 // -------------------------------------------------------------- launch ----
 
 struct Shape {
-    int engine, gmax, S, NW, R, C, smem, threads;
+    int engine, gmax, nmw, S, NW, R, C, PF, smem, threads;
 };
 
 int smem_bytes(const Shape &s, const Problem &pr)
@@ -277,14 +286,18 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         return ART_ERR_UNSUPPORTED;
     s.gmax = gmax_for(pr.G, s.engine);
     s.C = p->cluster_size;
+    s.nmw = (s.engine == art::kEngineMma && pr.B * pr.Hkv < di.sms) ? 4 : 1;
     const int tile = pr.page * pr.d * (int)elem_size(pr.dtype);
     const int units = pr.B * pr.Hkv;
+    // L2 prefetch ahead of the staged loads: off unless asked for (measured on
+    // the B200 it does not shorten the walk and it costs L2 space at high batch)
+    s.PF = p->prefetch > 0 ? p->prefetch : 0;
     // (compute warps, stages, window) in order of preference.  With at least
     // one unit per SM, two small CTAs per SM keep the most pages in flight;
     // with fewer units each unit is split over a cluster and needs a deeper
     // window to cover the latency from fetch to merged stop decision.
     static const int many_units[][3] = {{2, 2, 16}, {1, 2, 16}, {2, 2, 8}, {1, 2, 8}};
-    static const int few_units_large[][3] = {{2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
+    static const int few_units_large[][3] = {{4, 4, 24}, {2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
     static const int few_units_small[][3] = {{4, 8, 32}, {4, 8, 16}, {4, 4, 16}, {2, 4, 16}, {2, 2, 8},
                                              {1, 2, 8}};
     const int(*cand)[3];
@@ -294,7 +307,7 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         ncand = 4;
     } else if (tile >= 16384) {
         cand = few_units_large;
-        ncand = 5;
+        ncand = 6;
     } else {
         cand = few_units_small;
         ncand = 6;
@@ -309,7 +322,7 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         s.NW = NW;
         s.S = S;
         s.R = p->window ? p->window : cand[i][2];
-        s.threads = 32 * (1 + merge_warps(s.engine, pr.d, s.gmax) + NW);
+        s.threads = 32 * (1 + merge_warps(s.engine, pr.d, s.gmax, s.nmw) + NW);
         s.smem = smem_bytes(s, pr);
         if (s.smem <= di.smem_optin) {
             *out = s;
@@ -374,7 +387,7 @@ art_status_t launch(const art_params_t *p, art_stream_t stream)
     Shape s;
     if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
         return st;
-    KernelFn fn = pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax);
+    KernelFn fn = pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw);
     if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
         return st;
 
@@ -421,6 +434,7 @@ art_status_t launch(const art_params_t *p, art_stream_t stream)
     ka.S = s.S;
     ka.NW = s.NW;
     ka.R = s.R;
+    ka.PF = s.PF;
 
     CUtensorMap tmk, tmv;
     const bool swz = s.engine == art::kEngineMma;
@@ -450,6 +464,7 @@ art_status_t launch(const art_params_t *p, art_stream_t stream)
         p->info->stages = s.S;
         p->info->compute_warps = s.NW;
         p->info->window = s.R;
+        p->info->prefetch = s.PF;
         p->info->smem_bytes = s.smem;
     }
     if (cudaLaunchKernelEx(&cfg, fn, ka, tmk, tmv) != cudaSuccess) {

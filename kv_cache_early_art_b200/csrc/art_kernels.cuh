@@ -68,6 +68,7 @@ struct KernelArgs {
     int32_t *device_status;
     int32_t B, Hq, Hkv, G, num_pages, max_blocks;
     int32_t C, S, NW, R;                // cluster size, stages, compute warps, window
+    int32_t PF;                         // pages pulled into L2 ahead of the staged loads
     int64_t timeout_ns;
     int32_t debug_flags;
 };
@@ -97,7 +98,8 @@ __host__ __device__ inline Layout make_layout(int S, int NW, int R, int page, in
     L.pbuf_off = off;
     off += pbuf ? (uint32_t)(NW * page * gmax * 4) : 0u;
     L.red_off = off;
-    off += 2 * 4 * 33 * 4;  // merge-warp exchange: 2 batches x up to 4 warps x (32 sums + flag)
+    off += 2 * 4 * 34 * 4 + 16;  // merge-warp exchange: 2 batches x up to 4 warps x (32 sums, flag, norm),
+                                 // then the batch size merge warp 0 chose, per batch parity
     L.meta_off = off;
     off += 2 * S * 4;  // stage_j[S], stage_nv[S]
     off = round_up_u32(off, 8);
@@ -210,6 +212,23 @@ __device__ __forceinline__ void reduce_scatter32(float (&v)[32], int lane)
     }
 }
 
+// Butterfly reduce-scatter of 16 per-lane partial sums: afterwards v[0] of
+// lanes l and l+16 holds the warp-wide sum of entry l % 16.
+__device__ __forceinline__ void reduce_scatter16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int k = 8; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
+#pragma unroll
+        for (int i = 0; i < k; ++i) {
+            const float send = upper ? v[i] : v[i + k];
+            const float keep = upper ? v[i + k] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
 // Byte offset of bf16 element (t, d) in a K or V tile stored as d/64 column
 // slabs of [page][64] with the 128-byte TMA swizzle (16-byte chunk index
 // XOR row mod 8).
@@ -255,8 +274,11 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
     uint32_t issued = 0;        // stages handed out (pages, markers)
     uint32_t kphase = 0, vphase = 0;  // bit s: parity of the last phase armed on full_k[s] / full_v[s]
     uint32_t kused = 0, vused = 0;
-    uint32_t nfetched = 0;
+    uint32_t touched = 0;        // this CTA's walk steps whose page was read (loaded or prefetched)
     int batch_k0 = -1, my_lb = -1, my_pp = -1;
+    // L2 prefetch front: step k + PFS, PFS = ceil(PF / C) of this CTA's steps
+    const int PFS = (a.PF + C - 1) / C;
+    int pbatch_k0 = -1, my_plb = -1, my_ppp = -1;
     uint32_t ctrl_cache = 0;
     bool aborted = false;
 
@@ -311,6 +333,9 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
             }
         }
         go = __shfl_sync(0xffffffffu, go, 0);
+        // every branch below that holds a warp collective must be warp-uniform:
+        // give all lanes lane 0's view of the merged progress
+        ctrl_cache = __shfl_sync(0xffffffffu, ctrl_cache, 0);
         if (go == 0)
             break;
         if (go < 0) { aborted = true; break; }
@@ -352,10 +377,45 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         vphase ^= (vused >> s & 1u) ? (1u << s) : 0u;
         vused |= 1u << s;
         ++issued;
-        if (!bad)
-            ++nfetched;
-        else
+        if (bad)
             break;
+        touched = max(touched, (uint32_t)k + 1u);
+        // Keep the page PFS steps ahead warm in L2, within the window
+        // extended by PF: pages read past the stop stay below R + PF.
+        if (PFS > 0) {
+            const int kp = k + PFS;
+            const int jp = (int)rank + kp * C;
+            if (jp < N && (uint32_t)jp < ctrl_cache + (uint32_t)(R + a.PF)) {
+                if (pbatch_k0 < 0 || kp - pbatch_k0 >= 32) {
+                    pbatch_k0 = kp;
+                    const int jj = (int)rank + (kp + lane) * C;
+                    my_plb = -1;
+                    my_ppp = -1;
+                    if (jj < N) {
+                        my_plb = __ldg(bo + jj);
+                        if (my_plb >= 0 && my_plb < N)
+                            my_ppp = __ldg(pt + my_plb);
+                    }
+                }
+                const int plb = __shfl_sync(0xffffffffu, my_plb, kp - pbatch_k0);
+                const int ppp = __shfl_sync(0xffffffffu, my_ppp, kp - pbatch_k0);
+                if (plb >= 0 && plb < N && ppp >= 0 && ppp < a.num_pages) {
+                    if (lane == 0) {
+                        if constexpr (ENGINE == kEngineMma) {
+#pragma unroll
+                            for (int sb = 0; sb < D / 64; ++sb) {
+                                tma_prefetch_4d(tmk, sb * 64, 0, h, ppp);
+                                tma_prefetch_4d(tmv, sb * 64, 0, h, ppp);
+                            }
+                        } else {
+                            tma_prefetch_4d(tmk, 0, 0, h, ppp);
+                            tma_prefetch_4d(tmv, 0, 0, h, ppp);
+                        }
+                    }
+                    touched = max(touched, (uint32_t)kp + 1u);
+                }
+            }
+        }
     }
 
     if (!aborted) {
@@ -382,7 +442,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         }
     }
     if (lane == 0)
-        atom_add_cluster_u32(mapa(smem_u32((const void *)sh.fetched), 0), nfetched);
+        atom_add_cluster_u32(mapa(smem_u32((const void *)sh.fetched), 0), touched);
 }
 
 // ---- block engines -------------------------------------------------------------
@@ -570,18 +630,24 @@ struct MmaEngine {
         const uint32_t ku = smem_u32(kt), vu = smem_u32(vt);
 
         // scores, rows = tokens, columns = heads
-        float sacc[MT][4];
+        // (even and odd head-dim steps accumulate separately: shorter mma chains)
+        float sacc[MT][4], sodd[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sacc[mt][i] = sodd[mt][i] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 const int t = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int d = ks * 16 + (lane >> 4) * 8;
                 uint32_t a0, a1, a2, a3;
                 ldmatrix_x4(ku + swz128<PAGE>(t, d), a0, a1, a2, a3);
-                mma_bf16_16816(sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                mma_bf16_16816((ks & 1) ? sodd[mt] : sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sacc[mt][i] += sodd[mt][i];
         }
         const int g0 = 2 * c;
         float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};
@@ -781,11 +847,15 @@ struct MergeLayout<D, GMAX, kEngineMma> {  // tensor-core slots: vector v = dt*W
 // How the merge is split: NM warps share the output elements (vectors
 // [mw*NVW, mw*NVW+NVW) of every lane belong to merge warp mw); KB blocks are
 // folded per batch, with one scan lane per (block, head) pair.
-template <int D, int GMAX, int ENGINE>
+template <int D, int GMAX, int ENGINE, int NMW>
 struct MergeShape {
     using Lay = MergeLayout<D, GMAX, ENGINE>;
+    // at least one warp per 16 floats of output a lane keeps (registers), at
+    // most one per vector; all counts are powers of two
     static constexpr int TOT = Lay::NV * Lay::VW;
-    static constexpr int NM = TOT / 16 < 1 ? 1 : (TOT / 16 > 4 ? 4 : TOT / 16);
+    static constexpr int NMIN = TOT / 16 < 1 ? 1 : TOT / 16;
+    static constexpr int NM0 = NMW > NMIN ? NMW : NMIN;
+    static constexpr int NM = NM0 < Lay::NV ? NM0 : Lay::NV;
     static constexpr int NVW = Lay::NV / NM;
     static constexpr int KB = (32 / GMAX) < 8 ? (32 / GMAX) : 8;
     static_assert(Lay::NV % NM == 0, "merge split");
@@ -794,6 +864,11 @@ struct MergeShape {
 __device__ __forceinline__ void merge_barrier(int nthreads)
 {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void merge_barrier2(int nthreads)
+{
+    asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
 }
 
 // Folds block states into the running output in walk order, KB blocks per
@@ -806,12 +881,13 @@ __device__ __forceinline__ void merge_barrier(int nthreads)
 // reaching the same decision.  A stop inside a batch replays the batch up to
 // the stop from a snapshot, so the stop and the output are those of a
 // strictly sequential walk.
-template <int D, int GMAX, int ENGINE>
+template <int D, int GMAX, int ENGINE, int NMW>
 __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, int N, int mw)
 {
-    using MS = MergeShape<D, GMAX, ENGINE>;
+    using MS = MergeShape<D, GMAX, ENGINE, NMW>;
     using Lay = typename MS::Lay;
-    constexpr int NVW = MS::NVW, VW = Lay::VW, KB = MS::KB, NM = MS::NM;
+    constexpr int NVW = MS::NVW, VW = Lay::VW, VP = VW / 2, KB = MS::KB, NM = MS::NM;
+    static_assert(KB <= 8, "two partial sums per block in 16 lanes");
     const int lane = threadIdx.x & 31;
     const int G = a.G;
     const float eps_m = a.eps_m_arr ? a.eps_m_arr[b] : a.eps_m;
@@ -827,12 +903,13 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     // softmax scalars of head gl
     const int kl = lane / GMAX, gl = lane % GMAX;
     float Mx = -CUDART_INF_F, Lm = 0.f;
-    float o[NVW][VW];
+    // running output of this lane's elements, as packed fp32 pairs
+    uint64_t o[NVW][VP];
 #pragma unroll
     for (int i = 0; i < NVW; ++i)
 #pragma unroll
-        for (int e = 0; e < VW; ++e)
-            o[i][e] = 0.f;
+        for (int q = 0; q < VP; ++q)
+            o[i][q] = 0ull;
 
     int cnt = 0, stop = 0;
     bool failed = false;
@@ -842,50 +919,58 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
             failed = true;
     }
 
-    // fold batch block k (slot pointer sp) into this warp's slice of o, given
-    // this lane's u vectors uv; partial sums into pn, pd, pe
-    auto fold = [&](int k, float beta, const float (&uv)[NVW][VW], float &pn, float &pd, float &pe) {
-        float bsel[Lay::kTwoHeads ? 2 : NVW];
-        if constexpr (Lay::kTwoHeads) {
-            const int h0 = Lay::head(lane, 0, 0);
-            bsel[0] = __shfl_sync(0xffffffffu, beta, k * GMAX + h0);
-            bsel[1] = __shfl_sync(0xffffffffu, beta, k * GMAX + h0 + 1);
-        } else {
-#pragma unroll
-            for (int ii = 0; ii < NVW; ++ii)
-                bsel[ii] = __shfl_sync(0xffffffffu, beta, k * GMAX + vbase + ii);
-        }
-#pragma unroll
-        for (int ii = 0; ii < NVW; ++ii) {
-            if (!Lay::kTwoHeads && vbase + ii >= G)
-                continue;
-#pragma unroll
-            for (int e = 0; e < VW; ++e) {
-                const float bt = Lay::kTwoHeads ? bsel[e & 1] : bsel[Lay::kTwoHeads ? 0 : ii];
-                const float dl = bt * (uv[ii][e] - o[ii][e]);
-                pn = fmaf(o[ii][e], o[ii][e], pn);
-                pd = fmaf(o[ii][e], dl, pd);
-                pe = fmaf(dl, dl, pe);
-                o[ii][e] += dl;
-            }
-        }
-    };
-    auto load_u = [&](const float *sp, float (&uv)[NVW][VW]) {
+    auto load_u = [&](const float *sp, uint64_t (&uv)[NVW][VP]) {
 #pragma unroll
         for (int ii = 0; ii < NVW; ++ii) {
             const float *up = sp + u_off + Lay::off(lane, vbase + ii);
             if constexpr (VW == 4) {
                 const float4 x = *reinterpret_cast<const float4 *>(up);
-                uv[ii][0] = x.x; uv[ii][1] = x.y; uv[ii][2] = x.z; uv[ii][3] = x.w;
+                uv[ii][0] = pk2(x.x, x.y);
+                uv[ii][1] = pk2(x.z, x.w);
             } else {
                 const float2 x = *reinterpret_cast<const float2 *>(up);
-                uv[ii][0] = x.x; uv[ii][1] = x.y;
+                uv[ii][0] = pk2(x.x, x.y);
             }
         }
     };
+    // Fold batch block k into this warp's slice: Delta = beta (u - o),
+    // o += Delta; with sums, add o.Delta and |Delta|^2 of the slice to pd, pe.
+    auto fold = [&](int k, float beta, const uint64_t (&uv)[NVW][VP], float &pd, float &pe, bool sums) {
+        uint64_t bp[NVW];
+        if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads
+            const int h0 = Lay::head(lane, 0, 0);
+            const float b0 = __shfl_sync(0xffffffffu, beta, k * GMAX + h0);
+            const float b1 = __shfl_sync(0xffffffffu, beta, k * GMAX + h0 + 1);
+#pragma unroll
+            for (int ii = 0; ii < NVW; ++ii)
+                bp[ii] = pk2(b0, b1);
+        } else {  // vector i holds head i
+#pragma unroll
+            for (int ii = 0; ii < NVW; ++ii) {
+                const float bi = __shfl_sync(0xffffffffu, beta, k * GMAX + vbase + ii);
+                bp[ii] = (vbase + ii < G) ? pk2(bi, bi) : 0ull;
+            }
+        }
+        uint64_t sd = 0ull, se = 0ull;
+#pragma unroll
+        for (int ii = 0; ii < NVW; ++ii)
+#pragma unroll
+            for (int q = 0; q < VP; ++q) {
+                const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
+                if (sums) {
+                    sd = fma2(o[ii][q], dl, sd);
+                    se = fma2(dl, dl, se);
+                }
+                o[ii][q] = add2(o[ii][q], dl);
+            }
+        if (sums) {
+            pd = lo2(sd) + hi2(sd);
+            pe = lo2(se) + hi2(se);
+        }
+    };
     // fold blocks 0..kend of the batch starting at slot s0 (u loads one block ahead)
-    auto fold_batch = [&](int s0, int kend, float beta, float (&v)[32], bool sums) {
-        float ua[NVW][VW], ub[NVW][VW];
+    auto fold_batch = [&](int s0, int kend, float beta, float (&v)[16], bool sums) {
+        uint64_t ua[NVW][VP], ub[NVW][VP];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
 #pragma unroll
         for (int k = 0; k < KB; ++k) {
@@ -896,17 +981,17 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            float t0 = 0.f, t1 = 0.f, t2 = 0.f;
-            fold(k, beta, (k & 1) ? ub : ua, sums ? v[4 * k] : t0, sums ? v[4 * k + 1] : t1, sums ? v[4 * k + 2] : t2);
+            fold(k, beta, (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
         }
     };
 
     int s0 = 0;        // slot of the batch's first block, j0 % R
     uint32_t ph0 = 0;  // parity of that slot's phase, (j0 / R) & 1
-    for (int j0 = 0, batch = 0; !failed && stop == 0 && j0 < N; j0 += KB, ++batch) {
-        const int nb = min(KB, N - j0);
-        // 1. the batch's block states: lane k polls block j0 + k; a flagged
-        //    state (bad order or page entry upstream) ends the walk
+    for (int j0 = 0, batch = 0; !failed && stop == 0 && j0 < N; ++batch) {
+        const int nmax = min(KB, N - j0);
+        // 1. lane k polls block j0 + k until the whole batch has arrived.  A
+        //    flagged state (bad order or page entry upstream) ends the walk at
+        //    once: the blocks after it are never produced.
         int sk = s0 + (lane < KB ? lane : 0);
         uint32_t pk = ph0;
         if (sk >= a.R) {
@@ -915,16 +1000,24 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         }
         const float *spk = sh.ring + (size_t)sk * slot_floats;
         bool local_fail = false;
-        {
+        int nb = 0;
+        // Merge warp 0 alone polls; with several merge warps it hands the
+        // batch size (or a failure) to the others, so that all of them fold
+        // exactly the same blocks and meet at the same barriers.
+        if (mw == 0) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const bool arrived = lane >= nb || mbar_try_wait(sh.ready(sk, a.S), pk);
-                if (__any_sync(0xffffffffu, arrived && lane < nb && __float_as_uint(spk[0]) != 0u)) {
+                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk, a.S), pk);
+                if (__any_sync(0xffffffffu, arrived && __float_as_uint(spk[0]) != 0u)) {
                     local_fail = true;
                     break;
                 }
-                if (__all_sync(0xffffffffu, arrived))
+                // batches have fixed boundaries (multiples of KB), so the
+                // arithmetic, and the result, never depend on arrival timing
+                if (__all_sync(0xffffffffu, arrived || lane >= nmax)) {
+                    nb = nmax;
                     break;
+                }
                 if ((it & 7u) == 7u) {
                     int quit = 0;
                     if (lane == 0) {
@@ -946,12 +1039,21 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 }
             }
         }
-        float v[32];
+        if constexpr (NM > 1) {
+            volatile int *agreed = reinterpret_cast<volatile int *>(sh.red + 2 * 4 * 34) + (batch & 1);
+            if (mw == 0 && lane == 0)
+                *agreed = local_fail ? -1 : nb;
+            merge_barrier2(NM * 32);
+            const int v = *agreed;
+            local_fail = v < 0;
+            nb = v < 0 ? 0 : v;
+        }
+        float v[16];
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
+        for (int q = 0; q < 16; ++q)
             v[q] = 0.f;
-        float beta = 0.f;
-        float o0[NVW][VW];
+        float beta = 0.f, n0part = 0.f;
+        uint64_t o0[NVW][VP];
         if (!local_fail) {
             // 2. shares of the softmax mass: beta_(k,g) = w_k / (L_prev + w_0 + ... + w_k)
             float mk = -CUDART_INF_F, lk = 0.f;
@@ -978,72 +1080,93 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
             beta = Lam > 0.f ? w * rcp_approx(Lam) : 0.f;
             Lm = __shfl_sync(0xffffffffu, Lam, (nb - 1) * GMAX + gl);
             Mx = Mb;
-            // 3. fold the batch into this warp's slice
+            // 3. ||o||^2 before the batch, then fold the batch into this warp's slice
+            uint64_t n2 = 0ull;
 #pragma unroll
             for (int i = 0; i < NVW; ++i)
 #pragma unroll
-                for (int e = 0; e < VW; ++e)
-                    o0[i][e] = o[i][e];
+                for (int q = 0; q < VP; ++q) {
+                    o0[i][q] = o[i][q];
+                    n2 = fma2(o[i][q], o[i][q], n2);
+                }
+            n0part = lo2(n2) + hi2(n2);
             fold_batch(s0, nb - 1, beta, v, true);
-            reduce_scatter32(v, lane);  // lane 4k+q: quantity q of batch block k
         }
-        // 4. the slices meet; a failure anywhere ends the walk for every merge warp
-        float *red = sh.red + (batch & 1) * (NM * 33);
-        red[mw * 33 + lane] = v[0];
-        if (lane == 0)
-            reinterpret_cast<volatile int *>(red)[mw * 33 + 32] = local_fail ? 1 : 0;
+        // 4. lane 2k+q (and 2k+q+16): sum over the warp of quantity q of batch block k
+        reduce_scatter16(v, lane);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+            n0part += __shfl_xor_sync(0xffffffffu, n0part, off);
+        // the slices meet; a failure anywhere ends the walk for every merge warp
+        float *red = sh.red + (batch & 1) * (NM * 34);
+        red[mw * 34 + lane] = v[0];
+        if (lane == 0) {
+            reinterpret_cast<volatile int *>(red)[mw * 34 + 32] = local_fail ? 1 : 0;
+            red[mw * 34 + 33] = n0part;
+        }
         if constexpr (NM > 1)
             merge_barrier(NM * 32);
         else
             __syncwarp();
         bool any_fail = false;
-        float tot = 0.f;
+        float tot = 0.f, n0b = 0.f;
 #pragma unroll
         for (int w2 = 0; w2 < NM; ++w2) {
-            any_fail |= reinterpret_cast<volatile int *>(red)[w2 * 33 + 32] != 0;
-            tot += red[w2 * 33 + lane];
+            any_fail |= reinterpret_cast<volatile int *>(red)[w2 * 34 + 32] != 0;
+            tot += red[w2 * 34 + (lane & 15)];
+            n0b += red[w2 * 34 + 33];
         }
         if (any_fail) {
             failed = true;
             break;
         }
-        // 5. statistics of batch block k in lane 4k, then patience in walk order.
-        // ||o_j||^2 = ||o_{j-1}||^2 + 2 o_{j-1}.Delta + ||Delta||^2; the direction
-        // change uses the part of Delta orthogonal to o_{j-1}.
-        const int base = lane & ~3;
-        const float n0 = __shfl_sync(0xffffffffu, tot, base);
-        const float Dp = __shfl_sync(0xffffffffu, tot, base + 1);
-        const float Ep = __shfl_sync(0xffffffffu, tot, base + 2);
+        // 5. statistics of batch block k in lane 2k: ||o_{j-1}||^2 by a prefix
+        //    sum of t = 2 o_{j-1}.Delta + ||Delta||^2 over the batch's earlier
+        //    blocks; the direction change uses the part of Delta orthogonal to
+        //    o_{j-1}, so no near-equal O(1) numbers are subtracted.
+        const float Dp = tot;
+        const float Ep = __shfl_down_sync(0xffffffffu, tot, 1);
+        const float t = 2.f * Dp + Ep;
+        float pre = t;  // inclusive prefix over k in the even lanes 0..14
+#pragma unroll
+        for (int off = 2; off < 16; off <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, pre, off);
+            if ((lane & 15) >= off)
+                pre += u;
+        }
+        const float n0 = n0b + (pre - t);
+        const float n1sq = n0 + t;
         bool stable = false;
-        const float n1sq = n0 + 2.f * Dp + Ep;
         if (n0 > 0.f && n1sq > 0.f) {
-            const float r0 = sqrtf(n0), r1 = sqrtf(n1sq);
-            const float d_scale = fabsf(2.f * Dp + Ep) / ((r1 + r0) * r0);
-            const float x = r0 + Dp / r0;
-            const float y2 = fmaxf(Ep - (Dp / r0) * (Dp / r0), 0.f);
-            const float d_dir = x > 0.f ? y2 / (r1 * (r1 + x)) : 1.f - x / r1;
+            const float i0 = rsqrtf(n0), i1 = rsqrtf(n1sq);
+            const float r0 = n0 * i0, r1 = n1sq * i1;
+            const float d_scale = __fdividef(fabsf(t), (r1 + r0) * r0);
+            const float pr = Dp * i0;  // component of Delta along o_{j-1}
+            const float x = r0 + pr;
+            const float y2 = fmaxf(Ep - pr * pr, 0.f);
+            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : 1.f - x * i1;
             stable = (d_scale < eps_m) && (d_dir < eps_d);
         }
-        const uint32_t smask = __ballot_sync(0xffffffffu, stable && (lane & 3) == 0);
-        int kstop = -1;
-#pragma unroll
-        for (int k = 0; k < KB; ++k) {
-            const int j = j0 + k;
-            if (kstop < 0 && k < nb) {
-                if (j >= 1)
-                    cnt = (smask >> (4 * k) & 1u) ? cnt + 1 : 0;
-                if (cnt >= P && j + 1 >= minb)
-                    kstop = k;
-            }
-        }
+        // 6. patience over the batch, one lane per block: the counter after
+        //    block k is the run of stable blocks ending at k, plus the carried
+        //    count when the run reaches back to the batch start.  Block j = 0
+        //    of the walk is never compared, so it never counts as stable.
+        const bool stab_k = __shfl_sync(0xffffffffu, stable, 2 * (lane & 7)) && (j0 + (lane & 7) >= 1);
+        const uint32_t sbits = __ballot_sync(0xffffffffu, lane < nb && stab_k);
+        const int kq = lane & 7;
+        const uint32_t zeros = ~sbits & ((2u << kq) - 1u);  // unstable blocks at or before kq
+        const int run = zeros == 0u ? cnt + kq + 1 : kq - (31 - __clz(zeros));
+        const uint32_t hit = __ballot_sync(0xffffffffu, lane < nb && run >= P && j0 + kq + 1 >= minb);
+        const int kstop = hit ? __ffs(hit) - 1 : -1;
+        cnt = __shfl_sync(0xffffffffu, run, nb - 1);
         if (kstop >= 0) {
             stop = j0 + kstop + 1;
             if (kstop < nb - 1) {  // replay the batch up to the stop block
 #pragma unroll
                 for (int i = 0; i < NVW; ++i)
 #pragma unroll
-                    for (int e = 0; e < VW; ++e)
-                        o[i][e] = o0[i][e];
+                    for (int q = 0; q < VP; ++q)
+                        o[i][q] = o0[i][q];
                 fold_batch(s0, kstop, beta, v, false);
             }
         }
@@ -1052,7 +1175,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         // cannot overtake those reads.
         if (mw == 0 && lane == 0)
             st_relaxed_cluster_u32(ctrl_cl, stop ? (kStopBit | (uint32_t)stop) : (uint32_t)(j0 + nb));
-        s0 += KB;
+        j0 += nb;
+        s0 += nb;
         if (s0 >= a.R) {
             s0 -= a.R;
             ph0 ^= 1u;
@@ -1069,8 +1193,9 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         for (int e = 0; e < VW; ++e) {
             const int i = vbase + ii;
             const int g = Lay::head(lane, i, e);
+            const float val = (e & 1) ? hi2(o[ii][e >> 1]) : lo2(o[ii][e >> 1]);
             if (g < G && (Lay::kTwoHeads || i < G))
-                op[(int64_t)(h * G + g) * a.out_sh + Lay::dim(lane, i, e)] = failed ? 0.f : o[ii][e];
+                op[(int64_t)(h * G + g) * a.out_sh + Lay::dim(lane, i, e)] = failed ? 0.f : val;
         }
     if (mw == 0 && lane == 0)
         a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = failed ? -1 : stop;
@@ -1078,7 +1203,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 
 // ---- kernel ------------------------------------------------------------------------
 
-template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv)
@@ -1124,13 +1249,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     __syncthreads();
     cluster_sync();  // remote CTAs may now arrive on the leader's barriers
 
-    constexpr int NM = MergeShape<D, GMAX, ENGINE>::NM;
+    constexpr int NM = MergeShape<D, GMAX, ENGINE, NMW>::NM;
     if (N > 0 && !bad_len) {
         if (warp == 0)
             producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank);
         else if (warp <= NM) {
             if (rank == 0)
-                merge_role<D, GMAX, ENGINE>(a, sh, b, h, N, warp - 1);
+                merge_role<D, GMAX, ENGINE, NMW>(a, sh, b, h, N, warp - 1);
         } else
             compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM);
     } else if (rank == 0 && warp == 1) {

@@ -136,7 +136,8 @@ def test_ex_option_errors(art):
         setattr(p, name, a[key])
     lib = art.raw_library()
     for field, val in (("engine", 3), ("cluster_size", 17), ("stages", 9), ("stages", 1), ("window", 65),
-                       ("compute_warps", 7), ("window", 7), ("debug_flags", 2), ("timeout_ns", -1)):
+                       ("compute_warps", 7), ("window", 7), ("debug_flags", 2), ("timeout_ns", -1),
+                       ("prefetch", -2), ("prefetch", 65)):
         setattr(p, field, val)
         assert lib.art_decode_attention_ex(ctypes.byref(p), None) == -5, field
         setattr(p, field, 0)

@@ -39,7 +39,7 @@ def test_tiny_fp32_config(cuda_lib):
     assert status == 0
     s = parity.check(w, out, stop)
     assert s["canonical_mismatch"] == 0
-    assert_fetch_bound(w, stop, fetched, info["window"])
+    assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
 
 
 @pytest.mark.parametrize("engine", [1, 2])
@@ -48,7 +48,7 @@ def test_llama8b_b8_config(cuda_lib, engine):
     out, stop, fetched, status, info = run_gpu(cuda_lib, w, engine=engine)
     assert status == 0 and info["engine"] == engine
     parity.check(w, out, stop)
-    assert_fetch_bound(w, stop, fetched, info["window"])
+    assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
 
 
 SWEEP = []
@@ -75,7 +75,7 @@ def test_random_sweep(cuda_lib, seed, dtype, G, d, page, engine, cluster):
     assert status == 0
     assert info["cluster_size"] == cluster
     s = parity.check(w, out, stop)
-    assert_fetch_bound(w, stop, fetched, info["window"])
+    assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
     assert stop[3].tolist() == [0, 0] and (out[3] == 0).all()
 
 
@@ -191,7 +191,7 @@ def _full(art, name, seqs, engine=0):
     wc = parity.subset_sequences(w, seqs)
     idx = torch.as_tensor(seqs)
     s = parity.check(wc, out[idx], stop[idx])
-    assert_fetch_bound(w, stop, fetched, info["window"])
+    assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
     return s
 
 
