@@ -1,8 +1,8 @@
 """Benchmark: ART decode attention on one B200 (or N independent replicas).
 
-A step is one pass of the whole hot path over one decode batch: the default
-walk order is built on the device (sink block, then newest to oldest), then
-the ART walk runs for every (sequence, kv-head) unit.  The K/V cache is
+A step is one pass of the whole hot path over one decode batch: one launch
+of the ART walk for every (sequence, kv-head) unit, which builds the default
+walk order (sink block, then newest to oldest) on the fly in its producer.  The K/V cache is
 resident in HBM before timing starts; the L2 is flushed (a 512 MiB write)
 before every step, outside the step's events.
 
@@ -219,7 +219,7 @@ def config_for(name, w, gpus):
            "d": w.d, "page": w.page, "max_seq_len": int(w.seq_lens.max()),
            "params": ({"eps_m": p[0], "eps_d": p[1], "P": int(p[2]), "min_blocks": int(p[3])} if p else
                       "per-sequence"),
-           "order": "sink block, then newest to oldest (built on the device each step)",
+           "order": "sink block, then newest to oldest (built on the fly inside the walk)",
            "l2": "flushed before every step (512 MiB write, outside the step events)",
            "parallelism": f"replicas x{gpus} (independent batches, no collective)"}
     return cfg
@@ -249,7 +249,6 @@ def run_ours(args):
     block_bytes = 2 * page * d * esize            # K and V of one page of one kv head
     uni = w.uniform_params()
     stream = torch.cuda.current_stream(dev)
-    order = torch.empty_like(w.block_order)
     fetched = torch.zeros(B * Hkv, dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     out = torch.empty(B, w.Hq, d, dtype=torch.float32, device=dev)
@@ -257,30 +256,28 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
     def step(eps_off=False):
-        art.art_build_order_sink_recency(w.seq_lens, page, order)
         kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                   P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                   device_status=status, out=out, stop_block=stop)
-        return art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, order, w.seq_lens,
+        return art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
                                            eps_m=0.0, eps_d=0.0, want_info=True, **kw)
 
     def timed(n, eps_off=False):
-        """n steps; per step: flush, then [build order | walk] between events.
-        Returns per-step ms and walk-only ms."""
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        """n steps; per step: flush, then the walk between events.
+        Returns per-step ms (twice: the whole step is the walk)."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
         for i in range(n):
             flush.fill_(i)
             ev[i][0].record(stream)
-            art.art_build_order_sink_recency(w.seq_lens, page, order)
-            ev[i][1].record(stream)
             kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                       P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                       device_status=status, out=out, stop_block=stop)
-            art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, order, w.seq_lens,
+            art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
                                         eps_m=0.0, eps_d=0.0, **kw)
-            ev[i][2].record(stream)
+            ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        return ([e[0].elapsed_time(e[2]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev])
+        ms = [e[0].elapsed_time(e[1]) for e in ev]
+        return ms, ms
 
     _, _, info = step()
     for _ in range(max(args.warmup, 3)):
@@ -310,7 +307,7 @@ def run_ours(args):
     # ---- termination disabled: the same kernel as full attention ----
     for _ in range(2):
         step(eps_off=True)
-    f_step, f_walk = timed(max(3, args.steps // 2), eps_off=True)
+    f_step, f_walk = timed(max(3, args.steps // 4), eps_off=True)
     ms_full = sum(f_walk) / len(f_walk)
     full_consumed = int(stop.clamp(min=0).sum().item())
 
@@ -320,7 +317,7 @@ def run_ours(args):
     achieved = alg_bytes / (ms_walk / 1000.0) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "traffic": ncu_traffic(args.workload), "peak_kind": peak_kind,
-            "kernel": "art_walk_kernel (walk only; order builder excluded)",
+            "kernel": "art_walk_kernel (the whole step: the order is built inside it)",
             "algorithmic_bytes_per_launch": alg_bytes}
 
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
@@ -333,11 +330,11 @@ def run_ours(args):
             "hbm_frac_of_8tbs_spec": fetch_bytes / (ms_walk / 1000.0) / 1e9 / SPEC_HBM_GBS,
             "skip_frac_blocks": 1.0 - consumed / full_blocks,
             "fetch_waste_blocks": fetched_blocks - consumed,
-            "walk_ms": ms_walk, "order_ms": ms - ms_walk,
+            "walk_ms": ms_walk,
             "full_attention": {"walk_ms": ms_full, "kv_gbs": full_consumed * block_bytes / (ms_full / 1000.0) / 1e9,
                                "queries_per_s": B / (ms_full / 1000.0),
                                "art_speedup": ms_full / ms_walk},
-            "launch": info, "gpu_launches": 2 * args.steps,
+            "launch": info, "gpu_launches": args.steps,
             "roofline": roof, "clocks": clk.summary()}
 
     # ---- end to end through the public API: pinned host inputs in, results out ----
@@ -355,8 +352,7 @@ def run_ours(args):
             q_d.copy_(q_h, non_blocking=True)
             sl_d.copy_(sl_h, non_blocking=True)
             pt_d.copy_(pt_h, non_blocking=True)
-            art.art_build_order_sink_recency(sl_d, page, order)
-            art.art_decode_attention_ex(q_d, w.k_cache, w.v_cache, pt_d, order, sl_d, eps_m_per_seq=w.eps_m,
+            art.art_decode_attention_ex(q_d, w.k_cache, w.v_cache, pt_d, None, sl_d, eps_m_per_seq=w.eps_m,
                                         eps_d_per_seq=w.eps_d, P_per_seq=w.P, min_blocks_per_seq=w.min_blocks,
                                         out=out, stop_block=stop)
             out_h.copy_(out, non_blocking=True)
@@ -397,7 +393,7 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)

@@ -84,7 +84,10 @@ typedef enum {
  *  block_order [B, max_blocks] I32: logical block visited at walk step j; entries
  *                                   0..N_b-1 must be a permutation of 0..N_b-1 where
  *                                   N_b = ceil(seq_lens[b] / page).  Entries past
- *                                   N_b are never read.
+ *                                   N_b are never read.  May be NULL (or have NULL
+ *                                   data): the walk then takes the default order
+ *                                   [0, N_b-1, ..., 1] (sink block, then newest to
+ *                                   oldest), computed on the fly.
  *  seq_lens    [B] I32 (contiguous): tokens in the cache of sequence b.  Token
  *                                   lb*page + t of the sequence is row t of page
  *                                   page_table[b, lb]; rows past seq_lens[b] are masked.

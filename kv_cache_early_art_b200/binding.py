@@ -120,6 +120,7 @@ def _check(status: int, where: str):
 def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens, eps_m, eps_d, P, min_blocks,
                          out=None, stop_block=None, stream=None):
     """One ART decode-attention step (art_decode_attention in art.h).
+    block_order=None walks the default order (sink block, then newest first).
     Returns (out [B,Hq,d] fp32, stop_block [B,Hkv] int32)."""
     _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)
     B, Hq, d = q.shape
@@ -127,9 +128,11 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
         out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
     if stop_block is None:
         stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
-    ds = [descriptor(t) for t in (q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)]
-    st = _lib.art_decode_attention(*[ctypes.byref(x) for x in ds[:6]], float(eps_m), float(eps_d), int(P),
-                                   int(min_blocks), ctypes.byref(ds[6]), ctypes.byref(ds[7]), _stream(stream))
+    ds = [descriptor(t) if t is not None else None
+          for t in (q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)]
+    refs = [ctypes.byref(x) if x is not None else None for x in ds]
+    st = _lib.art_decode_attention(*refs[:6], float(eps_m), float(eps_d), int(P), int(min_blocks), refs[6],
+                                   refs[7], _stream(stream))
     _check(st, "art_decode_attention")
     return out, stop_block
 
@@ -155,7 +158,8 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p = ArtParams()
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("page_table", page_table),
                     ("block_order", block_order), ("seq_lens", seq_lens), ("out", out), ("stop_block", stop_block)):
-        setattr(p, name, descriptor(t))
+        if t is not None:           # block_order=None: the default order, built on the fly
+            setattr(p, name, descriptor(t))
     p.eps_m, p.eps_d, p.P, p.min_blocks = float(eps_m), float(eps_d), int(P), int(min_blocks)
     p.sm_scale = float(sm_scale)
     p.eps_m_per_seq = eps_m_per_seq.data_ptr() if eps_m_per_seq is not None else None

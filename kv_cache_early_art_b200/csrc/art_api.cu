@@ -34,15 +34,16 @@ art_status_t check_tensors(const art_params_t *p, Problem *pr)
 {
     const art_tensor_t *q = &p->q, *k = &p->k_cache, *v = &p->v_cache, *pt = &p->page_table,
                        *bo = &p->block_order, *sl = &p->seq_lens, *o = &p->out, *st = &p->stop_block;
-    if (is_null(q) || is_null(k) || is_null(v) || is_null(pt) || is_null(bo) || is_null(sl) || is_null(o) ||
-        is_null(st))
+    // block_order may be absent (NULL data): the default order is then built on the fly
+    const bool has_order = bo->data != nullptr;
+    if (is_null(q) || is_null(k) || is_null(v) || is_null(pt) || is_null(sl) || is_null(o) || is_null(st))
         return ART_ERR_NULL;
-    if (q->ndim != 3 || k->ndim != 4 || v->ndim != 4 || pt->ndim != 2 || bo->ndim != 2 || sl->ndim != 1 ||
-        o->ndim != 3 || st->ndim != 2)
+    if (q->ndim != 3 || k->ndim != 4 || v->ndim != 4 || pt->ndim != 2 || (has_order && bo->ndim != 2) ||
+        sl->ndim != 1 || o->ndim != 3 || st->ndim != 2)
         return ART_ERR_SHAPE;
     if (q->dtype != ART_F32 && q->dtype != ART_BF16)
         return ART_ERR_DTYPE;
-    if (k->dtype != q->dtype || v->dtype != q->dtype || pt->dtype != ART_I32 || bo->dtype != ART_I32 ||
+    if (k->dtype != q->dtype || v->dtype != q->dtype || pt->dtype != ART_I32 || (has_order && bo->dtype != ART_I32) ||
         sl->dtype != ART_I32 || o->dtype != ART_F32 || st->dtype != ART_I32)
         return ART_ERR_DTYPE;
     const int64_t B = q->shape[0], Hq = q->shape[1], d = q->shape[2];
@@ -56,15 +57,15 @@ art_status_t check_tensors(const art_params_t *p, Problem *pr)
             return ART_ERR_SHAPE;
     if (k->shape[3] != d || Hq % Hkv != 0)
         return ART_ERR_SHAPE;
-    if (pt->shape[0] != B || bo->shape[0] != B || pt->shape[1] != bo->shape[1] || pt->shape[1] <= 0 ||
-        pt->shape[1] > (int64_t)INT32_MAX / 256 || sl->shape[0] != B)
+    if (pt->shape[0] != B || (has_order && (bo->shape[0] != B || pt->shape[1] != bo->shape[1])) ||
+        pt->shape[1] <= 0 || pt->shape[1] > (int64_t)INT32_MAX / 256 || sl->shape[0] != B)
         return ART_ERR_SHAPE;
     if (o->shape[0] != B || o->shape[1] != Hq || o->shape[2] != d || st->shape[0] != B || st->shape[1] != Hkv)
         return ART_ERR_SHAPE;
     // contiguity and alignment the kernels rely on
     const int64_t es = elem_size(q->dtype);
     if (q->stride[2] != 1 || k->stride[3] != 1 || v->stride[3] != 1 || pt->stride[1] != 1 ||
-        bo->stride[1] != 1 || sl->stride[0] != 1 || o->stride[2] != 1)
+        (has_order && bo->stride[1] != 1) || sl->stride[0] != 1 || o->stride[2] != 1)
         return ART_ERR_SHAPE;
     if (!aligned(q->data, 16) || (q->stride[0] * es) % 16 || (q->stride[1] * es) % 16 || q->stride[0] < 0 ||
         q->stride[1] < 0)
@@ -76,7 +77,7 @@ art_status_t check_tensors(const art_params_t *p, Problem *pr)
             if (c->stride[i] <= 0 || (c->stride[i] * es) % 16 || c->stride[i] * es >= (int64_t)1 << 40)
                 return ART_ERR_SHAPE;
     }
-    if (!aligned(pt->data, 4) || !aligned(bo->data, 4) || !aligned(sl->data, 4) || !aligned(o->data, 4) ||
+    if (!aligned(pt->data, 4) || (has_order && !aligned(bo->data, 4)) || !aligned(sl->data, 4) || !aligned(o->data, 4) ||
         !aligned(st->data, 4))
         return ART_ERR_SHAPE;
     const int64_t G = Hq / Hkv;
@@ -491,7 +492,7 @@ art_status_t art_decode_attention(const art_tensor_t *q, const art_tensor_t *k_c
                                   int32_t min_blocks, art_tensor_t *out, art_tensor_t *stop_block,
                                   art_stream_t stream)
 {
-    if (!q || !k_cache || !v_cache || !page_table || !block_order || !seq_lens || !out || !stop_block)
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out || !stop_block)
         return ART_ERR_NULL;
     art_params_t p;
     std::memset(&p, 0, sizeof p);
@@ -499,7 +500,8 @@ art_status_t art_decode_attention(const art_tensor_t *q, const art_tensor_t *k_c
     p.k_cache = *k_cache;
     p.v_cache = *v_cache;
     p.page_table = *page_table;
-    p.block_order = *block_order;
+    if (block_order)
+        p.block_order = *block_order;  // else zeroed: the default order
     p.seq_lens = *seq_lens;
     p.out = *out;
     p.stop_block = *stop_block;

@@ -265,7 +265,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
     const int lane = threadIdx.x & 31;
     const int S = a.S, R = a.R, C = a.C;
     const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
-    const int32_t *bo = a.block_order + (int64_t)b * a.bo_sb;
+    const int32_t *bo = a.block_order ? a.block_order + (int64_t)b * a.bo_sb : nullptr;
     const int32_t *pt = a.page_table + (int64_t)b * a.pt_sb;
     if (lane == 0) {
         prefetch_tensormap(tmk);
@@ -299,7 +299,8 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
             my_lb = -1;
             my_pp = -1;
             if (jj < N) {
-                my_lb = __ldg(bo + jj);
+                // no order given: the sink block, then newest to oldest
+                my_lb = a.block_order ? __ldg(bo + jj) : (jj == 0 ? 0 : N - jj);
                 if (my_lb >= 0 && my_lb < N)
                     my_pp = __ldg(pt + my_lb);
             }
@@ -392,7 +393,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
                     my_plb = -1;
                     my_ppp = -1;
                     if (jj < N) {
-                        my_plb = __ldg(bo + jj);
+                        my_plb = a.block_order ? __ldg(bo + jj) : (jj == 0 ? 0 : N - jj);
                         if (my_plb >= 0 && my_plb < N)
                             my_ppp = __ldg(pt + my_plb);
                     }

@@ -110,6 +110,25 @@ def test_sink_order_builder(cuda_lib):
     assert torch.equal(order.cpu(), sink_recency_order(N, 70))
 
 
+@pytest.mark.parametrize("cluster", [1, 2])
+def test_default_order_on_the_fly(cuda_lib, cluster):
+    """No block_order: the walk builds sink-then-newest-first itself, and the
+    result equals the same walk given that order explicitly, bit for bit."""
+    w = make_custom(B=4, Hq=16, Hkv=4, d=128, page=64, dtype="bf16", seq_lens=[3000, 64, 777, 1],
+                    seed=21, planted=3, planted_gain=5.0, order="sink_recency", eps_m=5e-3, eps_d=5e-4, P=2)
+    g = w.to("cuda")
+    kw = dict(eps_m=5e-3, eps_d=5e-4, P=2, min_blocks=1, cluster_size=cluster)
+    out0, stop0 = cuda_lib.art_decode_attention_ex(g.q, g.k_cache, g.v_cache, g.page_table, None, g.seq_lens, **kw)
+    out1, stop1 = cuda_lib.art_decode_attention_ex(g.q, g.k_cache, g.v_cache, g.page_table, g.block_order,
+                                                   g.seq_lens, **kw)
+    out2, stop2 = cuda_lib.art_decode_attention(g.q, g.k_cache, g.v_cache, g.page_table, None, g.seq_lens,
+                                                5e-3, 5e-4, 2, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(stop0, stop1) and torch.equal(out0, out1)
+    assert torch.equal(stop0, stop2) and torch.equal(out0, out2)
+    parity.check(w, out0, stop0)
+
+
 def test_strided_cache_layout(cuda_lib):
     """Cache stored as [num_pages, page, Hkv, d] and viewed with strides."""
     w = make_custom(B=2, Hq=8, Hkv=2, d=128, page=64, dtype="bf16", seq_lens=[900, 300], seed=9,
