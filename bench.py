@@ -8,6 +8,7 @@ before every step, outside the step's events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+    python bench.py --table all      # every workload: ART, eps=0 and ablations
 
 Under torchrun each rank runs its own batch of the same shape (weak scaling,
 no collective on the data path); rank 0 prints one JSON line.
@@ -184,7 +185,19 @@ def time_oracle(w_cpu, budget_s: float):
     return w_cpu.B * reps / el, ncores, reps, el
 
 
+def one_sequence(w, b):
+    """Sequence b of a CPU workload, sharing its caches (the oracle's sample)."""
+    v = w.to("cpu")
+    sl = slice(b, b + 1)
+    v.q, v.page_table, v.block_order, v.seq_lens = w.q[sl], w.page_table[sl], w.block_order[sl], w.seq_lens[sl]
+    v.eps_m, v.eps_d, v.P, v.min_blocks = w.eps_m[sl], w.eps_d[sl], w.P[sl], w.min_blocks[sl]
+    return v
+
+
 def run_reference(args):
+    """The CPU oracle timed on the host cores; each step is a bounded sample of
+    the workload: one sequence (one decode query, all its kv heads), cycling
+    through the batch."""
     ws, rank, local = dist_env()
     if rank != 0:
         return 0
@@ -192,16 +205,17 @@ def run_reference(args):
     w = make_workload(args.workload, seed=replica_seed(0), device="cpu")
     import oracle
     ncores = os.cpu_count() or 1
-    for _ in range(args.warmup):
-        oracle.run(w, nthreads=ncores)
+    samples = [one_sequence(w, b) for b in range(w.B)]
+    for i in range(args.warmup):
+        oracle.run(samples[i % w.B], nthreads=ncores)
     times = []
-    for _ in range(args.steps):
+    for i in range(args.steps):
         t0 = time.perf_counter()
-        oracle.run(w, nthreads=ncores)
+        oracle.run(samples[i % w.B], nthreads=ncores)
         times.append(time.perf_counter() - t0)
     ms = 1000.0 * sum(times) / len(times)
-    value = w.B / (ms / 1000.0)
-    sample = f"whole {args.workload} batch ({w.B} queries, all {w.B * w.Hkv} units) per step"
+    value = 1.0 / (ms / 1000.0)
+    sample = f"one {args.workload} sequence per step (1 query, its {w.Hkv} kv-head units), cycling the batch"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -390,6 +404,84 @@ def run_ours(args):
     return 0
 
 
+def run_table(args):
+    """Every named workload (and two pruned-cache variants) with ART, the same
+    kernel with termination disabled (eps = 0), and the ablations of the ART
+    explainer's section 4 (scale only, direction only, no patience): walk time,
+    blocks consumed and skipped, pages fetched, GB/s.  One JSON line per row,
+    then a markdown table."""
+    import torch
+
+    import kv_cache_early_art_b200 as art
+    from kv_cache_early_art_b200.workloads import CONFIGS, make_workload, streaming_subset
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    peak, _ = measured_peaks()
+    inf = float("inf")
+    rows = []
+
+    def measure(w, label, em, ed, P):
+        out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+        stop = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev)
+        fetched = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        kw = dict(eps_m_per_seq=em, eps_d_per_seq=ed, P_per_seq=P, min_blocks_per_seq=w.min_blocks,
+                  blocks_fetched=fetched, device_status=status, out=out, stop_block=stop)
+        call = lambda: art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, w.block_order,
+                                                   w.seq_lens, **kw)
+        call()
+        ts = []
+        for i in range(args.table_reps):
+            flush.fill_(i)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        ms = ts[len(ts) // 2]
+        assert int(status.item()) == 0
+        N = w.n_blocks().to(dev)
+        total = int(N.sum().item()) * w.Hkv
+        used = int(stop.clamp(min=0).sum().item())
+        bb = 2 * w.page * w.d * w.k_cache.element_size()
+        row = {"workload": w.name, "variant": label, "ms": ms, "queries_per_s": w.B / (ms / 1e3),
+               "blocks": total, "consumed": used, "skip_frac": 1.0 - used / max(total, 1),
+               "fetched": int(fetched.sum().item()), "gbs": used * bb / (ms / 1e3) / 1e9,
+               "hbm_frac": used * bb / (ms / 1e3) / 1e9 / peak}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+
+    names = list(CONFIGS) if args.table == "all" else args.table.split(",")
+    for name in names:
+        base = make_workload(name, device=dev)
+        variants = [base]
+        if name in ("llama8b_b32", "qwen7b_b4"):   # a StreamingLLM-style pruned cache: sink + last 64 pages
+            variants.append(streaming_subset(base, window_blocks=64))
+        for w in variants:
+            B = w.B
+            ones = torch.ones(B, dtype=torch.int32, device=dev)
+            full = lambda v: torch.full((B,), v, dtype=torch.float32, device=dev)
+            measure(w, "ART", w.eps_m, w.eps_d, w.P)
+            measure(w, "full (eps=0)", full(0.0), full(0.0), w.P)
+            measure(w, "scale only", w.eps_m, full(inf), w.P)
+            measure(w, "direction only", full(inf), w.eps_d, w.P)
+            measure(w, "no patience (P=1)", w.eps_m, w.eps_d, ones)
+        del base, variants
+        torch.cuda.empty_cache()
+    print("| workload | variant | walk ms | queries/s | blocks consumed / total | skipped | pages fetched | GB/s | of HBM |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r['workload']} | {r['variant']} | {r['ms']:.4f} | {r['queries_per_s']:.0f} | "
+              f"{r['consumed']} / {r['blocks']} | {100 * r['skip_frac']:.1f} % | {r['fetched']} | "
+              f"{r['gbs']:.0f} | {100 * r['hbm_frac']:.1f} % |")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -400,7 +492,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--table", default=None, help="'all' or comma-separated workloads: per-workload table")
+    ap.add_argument("--table-reps", type=int, default=20)
     args = ap.parse_args(argv)
+    if args.table:
+        return run_table(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -26,14 +26,18 @@ it):
                     ragged L uniform in [1024, 16384], per-sequence patience
                     in {1,2,4} and eps_m in {1e-4, 1e-3} (eps_d = eps_m/10).
 
-Draw order (one ``torch.Generator`` seeded once; fixed so that the same seed
-always gives the same bits on a given device):
+Draw order (fixed, so that the same seed always gives the same bits on a
+given device):
 
-1. sequence lengths (ragged workloads only), then per-sequence P and eps_m;
+1. ragged workloads only: sequence lengths, then per-sequence P and eps_m,
+   from a CPU ``torch.Generator`` seeded with ``seed ^ 0x5EED``;
+then, from one ``torch.Generator`` on the target device seeded with ``seed``:
 2. q ~ N(0,1) of shape [B, Hq, d];
 3. a permutation of the physical pages (random page tables only);
 4. planted positions, per sequence (planted workloads only);
-5. per sequence b: K noise [Hkv, L_b, d], then V [Hkv, L_b, d].
+5. per sequence b: K noise [Hkv, L_b, d], then V [Hkv, L_b, d];
+6. ``order="random"`` only: a permutation per sequence from a CPU generator
+   seeded with ``seed * 7919 + b``.
 
 Keys for recency workloads: k_t = noise_t + alpha_t * q_hat_grp with
 alpha_t = 2 * (1 + age)^-0.5, age = L_b - 1 - t, and q_hat_grp the unit
@@ -49,7 +53,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["Workload", "CONFIGS", "make_workload", "make_custom", "sink_recency_order"]
+__all__ = ["Workload", "CONFIGS", "make_workload", "make_custom", "sink_recency_order", "streaming_subset"]
 
 
 @dataclass
@@ -304,3 +308,41 @@ def make_workload(name: str, seed: int = 0, device="cpu") -> Workload:
                     page_table=c["page_table"], eps_m=em, eps_d=ed, P=P,
                     min_blocks=c["min_blocks"], device=device, name=name)
     return w
+
+
+def streaming_subset(w: Workload, window_blocks: int, sink_blocks: int = 1, name: str = None) -> Workload:
+    """The same cache seen through a StreamingLLM-style pruning policy: per
+    sequence only its first ``sink_blocks`` pages (attention sinks) and its
+    last ``window_blocks`` pages are kept.  The kept pages are re-listed in a
+    compacted page table (sinks first, then the window oldest to newest), so
+    the pruned sequence is an ordinary paged sequence whose only partial page
+    is its last; ``seq_lens`` shrink accordingly and the walk order becomes
+    the default one of the compacted sequence.  K, V and q are shared with
+    ``w`` (no copy).  This is how ART composes with a pruned cache (ART
+    explainer, section 2.4: an orthogonal layer over the kept blocks)."""
+    N = w.n_blocks().cpu()
+    L = w.seq_lens.cpu().to(torch.int64)
+    pt = w.page_table.cpu()
+    B = w.B
+    keep_n = torch.zeros(B, dtype=torch.int64)
+    new_len = torch.zeros(B, dtype=torch.int64)
+    rows = []
+    for b in range(B):
+        n, l = int(N[b]), int(L[b])
+        if n <= sink_blocks + window_blocks:
+            blocks = list(range(n))
+        else:
+            blocks = list(range(sink_blocks)) + list(range(n - window_blocks, n))
+        rows.append(pt[b, blocks] if blocks else pt[b, :0])
+        keep_n[b] = len(blocks)
+        last = l - (n - 1) * w.page if n else 0          # tokens in the sequence's last page
+        new_len[b] = (len(blocks) - 1) * w.page + last if blocks else 0
+    mb = max(1, int(keep_n.max()))
+    new_pt = torch.full((B, mb), -1, dtype=torch.int32)
+    for b in range(B):
+        new_pt[b, :int(keep_n[b])] = rows[b].to(torch.int32)
+    dev = w.q.device
+    order = sink_recency_order(keep_n, mb)
+    return Workload(name or f"{w.name}_stream{window_blocks}", w.q, w.k_cache, w.v_cache, new_pt.to(dev),
+                    order.to(dev), new_len.to(torch.int32).to(dev), w.eps_m, w.eps_d, w.P, w.min_blocks,
+                    w.page, dict(w.meta, pruned=f"sinks {sink_blocks} + window {window_blocks} pages"))

@@ -129,6 +129,20 @@ def test_default_order_on_the_fly(cuda_lib, cluster):
     parity.check(w, out0, stop0)
 
 
+def test_over_pruned_cache(cuda_lib):
+    """ART on a StreamingLLM-style pruned cache (sink page + recent window,
+    compacted page table): parity with the oracle on the same pruned view."""
+    from kv_cache_early_art_b200.workloads import streaming_subset
+    base = make_custom(B=3, Hq=16, Hkv=4, d=128, page=64, dtype="bf16", seq_lens=[5000, 700, 130], seed=22,
+                       planted=4, planted_gain=5.0, eps_m=5e-3, eps_d=5e-4, P=2)
+    w = streaming_subset(base, window_blocks=16)
+    assert w.n_blocks().tolist() == [17, 11, 3]
+    out, stop, fetched, status, info = run_gpu(cuda_lib, w)
+    assert status == 0
+    parity.check(w, out, stop)
+    assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
+
+
 def test_strided_cache_layout(cuda_lib):
     """Cache stored as [num_pages, page, Hkv, d] and viewed with strides."""
     w = make_custom(B=2, Hq=8, Hkv=2, d=128, page=64, dtype="bf16", seq_lens=[900, 300], seed=9,
