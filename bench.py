@@ -8,7 +8,7 @@ before every step, outside the step's events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-cpu-baseline] [--no-e2e]
-    python bench.py --table all      # every workload: ART, eps=0 and ablations
+    python bench.py --table all      # every workload: ART, eps=0, ablations, importance order
 
 Under torchrun each rank runs its own batch of the same shape (weak scaling,
 no collective on the data path); rank 0 prints one JSON line.
@@ -422,28 +422,40 @@ def run_table(args):
     inf = float("inf")
     rows = []
 
-    def measure(w, label, em, ed, P):
-        out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
-        stop = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev)
-        fetched = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device=dev)
-        status = torch.zeros(1, dtype=torch.int32, device=dev)
-        kw = dict(eps_m_per_seq=em, eps_d_per_seq=ed, P_per_seq=P, min_blocks_per_seq=w.min_blocks,
-                  blocks_fetched=fetched, device_status=status, out=out, stop_block=stop)
-        call = lambda: art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, w.block_order,
-                                                   w.seq_lens, **kw)
-        call()
+    def median_ms(fn):
         ts = []
         for i in range(args.table_reps):
             flush.fill_(i)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
-            call()
+            fn()
             b.record()
             torch.cuda.synchronize(dev)
             ts.append(a.elapsed_time(b))
         ts.sort()
-        ms = ts[len(ts) // 2]
+        return ts[len(ts) // 2]
+
+    def measure(w, label, em, ed, P, importance=None):
+        """importance = (summary, scores, order): the order is rebuilt from the
+        page summaries inside the timed region, before the walk."""
+        out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+        stop = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev)
+        fetched = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        kw = dict(eps_m_per_seq=em, eps_d_per_seq=ed, P_per_seq=P, min_blocks_per_seq=w.min_blocks,
+                  blocks_fetched=fetched, device_status=status, out=out, stop_block=stop)
+        order = w.block_order if importance is None else importance[2]
+
+        def call():
+            if importance is not None:
+                art.art_build_order_importance(w.q, importance[0], w.page_table, w.seq_lens, w.page,
+                                               block_scores=importance[1], block_order=importance[2],
+                                               device_status=status)
+            art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, order, w.seq_lens, **kw)
+
+        call()
+        ms = median_ms(call)
         assert int(status.item()) == 0
         N = w.n_blocks().to(dev)
         total = int(N.sum().item()) * w.Hkv
@@ -455,6 +467,7 @@ def run_table(args):
                "hbm_frac": used * bb / (ms / 1e3) / 1e9 / peak}
         rows.append(row)
         print(json.dumps(row), flush=True)
+        return row
 
     names = list(CONFIGS) if args.table == "all" else args.table.split(",")
     for name in names:
@@ -471,6 +484,17 @@ def run_table(args):
             measure(w, "scale only", w.eps_m, full(inf), w.P)
             measure(w, "direction only", full(inf), w.eps_d, w.P)
             measure(w, "no patience (P=1)", w.eps_m, w.eps_d, ones)
+            # importance-first order: page summaries kept beside the cache (built
+            # once, timed apart), the order rebuilt every step inside the timing
+            summ = art.art_page_summary(w.k_cache, w.page_table, w.seq_lens, dtype=torch.bfloat16)
+            sum_ms = median_ms(lambda: art.art_page_summary(w.k_cache, w.page_table, w.seq_lens, summ))
+            bufs = (summ, torch.empty(B, w.max_blocks, dtype=torch.float32, device=dev),
+                    torch.empty(B, w.max_blocks, dtype=torch.int32, device=dev))
+            order_ms = median_ms(lambda: art.art_build_order_importance(
+                w.q, summ, w.page_table, w.seq_lens, w.page, block_scores=bufs[1], block_order=bufs[2]))
+            row = measure(w, "ART, importance order", w.eps_m, w.eps_d, w.P, importance=bufs)
+            row.update(summary_ms=sum_ms, order_ms=order_ms)
+            print(json.dumps({"workload": w.name, "summary_ms": sum_ms, "order_ms": order_ms}), flush=True)
         del base, variants
         torch.cuda.empty_cache()
     print("| workload | variant | walk ms | queries/s | blocks consumed / total | skipped | pages fetched | GB/s | of HBM |")
@@ -479,6 +503,12 @@ def run_table(args):
         print(f"| {r['workload']} | {r['variant']} | {r['ms']:.4f} | {r['queries_per_s']:.0f} | "
               f"{r['consumed']} / {r['blocks']} | {100 * r['skip_frac']:.1f} % | {r['fetched']} | "
               f"{r['gbs']:.0f} | {100 * r['hbm_frac']:.1f} % |")
+    print()
+    print("| workload | page summaries (once per page fill) ms | importance order build ms (inside the row above) |")
+    print("|---|---|---|")
+    for r in rows:
+        if "summary_ms" in r:
+            print(f"| {r['workload']} | {r['summary_ms']:.4f} | {r['order_ms']:.4f} |")
     return 0
 
 

@@ -163,6 +163,62 @@ art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
 art_status_t art_build_order_sink_recency(const art_tensor_t *seq_lens, int32_t page,
                                           art_tensor_t *block_order, art_stream_t stream);
 
+/*
+ * Importance-first traversal (section 2.4 names "importance-first" next to
+ * "recency-first" as an order ART can run over, with block 0 kept first; the
+ * explainer gives no importance estimate, so the one below is this
+ * library's own).  Two calls:
+ *
+ * art_page_summary -- the summary of every page a sequence references: the
+ * mean of the page's valid keys, per kv-head,
+ *     summary[p, h, :] = (1/n) sum_{t < n} k_cache[p, h, t, :],
+ * where p = page_table[b, j] for j < N_b and n = min(page, seq_lens[b] -
+ * j*page).  Sums are fp32; the mean is rounded once to the summary's
+ * type.  It reads the whole referenced K cache once: call it when
+ * pages are filled (a page whose tokens do not change keeps its summary),
+ * not per decode step.
+ *   k_cache    [num_pages, Hkv, page, d] F32|BF16, d contiguous, 16-byte
+ *              aligned base and strides (the layout art_decode_attention
+ *              takes); d a power of two from 16 to 256.
+ *   page_table [B, max_blocks] I32, seq_lens [B] I32 (as for the walk).
+ *   summary    [num_pages, Hkv, d] F32|BF16 out, d contiguous, 16-byte
+ *              aligned base and strides.  Pages no sequence references are
+ *              not written.  A page referenced by several sequences must
+ *              hold the same number of valid tokens in each.
+ *   device_status  device [1] or NULL: a page-table entry outside
+ *              [0, num_pages), or N_b > max_blocks, stores ART_ERR_BAD_INDEX
+ *              there; the bad page is skipped.
+ *
+ * art_build_order_importance -- scores every block and writes the walk order
+ * block 0 first, then blocks 1..N_b-1 by decreasing score, equal scores
+ * newest (larger index) first, then -1 up to max_blocks.  The score of
+ * block j of sequence b is the page mean of the attention logit summed over
+ * all query heads (query head i reads kv-head i / G):
+ *     block_scores[b, j] = sm_scale * sum_i q[b, i, :] . summary[page_table[b, j], i / G, :]
+ * (fp32; -0 is stored as +0; -inf for j >= N_b).  The order is the exact
+ * sort of the stored fp32 scores, so it is a permutation of 0..N_b-1 for any
+ * input, NaN scores included, and is bitwise reproducible.
+ *   q            [B, Hq, d] F32|BF16, d contiguous, 16-byte aligned base and
+ *                strides; Hq a multiple of Hkv; Hkv*d at most 16384.
+ *   summary      as written by art_page_summary (F32|BF16).
+ *   page_table   [B, max_blocks] I32; seq_lens [B] I32; page > 0.
+ *   sm_scale     the logit scale; <= 0 selects 1/sqrt(d).
+ *   block_scores [B, max_blocks] F32 out, last dimension contiguous.
+ *   block_order  [B, max_blocks] I32 out, last dimension contiguous; feed it
+ *                to art_decode_attention.
+ *   device_status  as above (bad page entries get a NaN score).
+ * Both calls are asynchronous on the stream and allocate nothing.
+ */
+art_status_t art_page_summary(const art_tensor_t *k_cache, const art_tensor_t *page_table,
+                              const art_tensor_t *seq_lens, art_tensor_t *summary,
+                              int32_t *device_status, art_stream_t stream);
+
+art_status_t art_build_order_importance(const art_tensor_t *q, const art_tensor_t *summary,
+                                        const art_tensor_t *page_table, const art_tensor_t *seq_lens,
+                                        int32_t page, float sm_scale, art_tensor_t *block_scores,
+                                        art_tensor_t *block_order, int32_t *device_status,
+                                        art_stream_t stream);
+
 /* Static description of a status code. */
 const char *art_strerror(art_status_t status);
 

@@ -68,6 +68,11 @@ _lib.art_decode_attention_ex.argtypes = [_P(ArtParams), ctypes.c_void_p]
 _lib.art_decode_attention_ex.restype = ctypes.c_int
 _lib.art_build_order_sink_recency.argtypes = [_P(ArtTensor), ctypes.c_int32, _P(ArtTensor), ctypes.c_void_p]
 _lib.art_build_order_sink_recency.restype = ctypes.c_int
+_lib.art_page_summary.argtypes = [_P(ArtTensor)] * 4 + [ctypes.c_void_p, ctypes.c_void_p]
+_lib.art_page_summary.restype = ctypes.c_int
+_lib.art_build_order_importance.argtypes = [_P(ArtTensor)] * 4 + [ctypes.c_int32, ctypes.c_float] + [
+    _P(ArtTensor)] * 2 + [ctypes.c_void_p, ctypes.c_void_p]
+_lib.art_build_order_importance.restype = ctypes.c_int
 _lib.art_strerror.argtypes = [ctypes.c_int]
 _lib.art_strerror.restype = ctypes.c_char_p
 _lib.art_version.argtypes = []
@@ -192,6 +197,47 @@ def art_build_order_sink_recency(seq_lens, page, block_order=None, max_blocks=No
     st = _lib.art_build_order_sink_recency(ctypes.byref(a), int(page), ctypes.byref(b), _stream(stream))
     _check(st, "art_build_order_sink_recency")
     return block_order
+
+
+def _status_ptr(device_status):
+    if device_status is None:
+        return None
+    _need_cuda(device_status)
+    if device_status.dtype != torch.int32 or device_status.numel() < 1:
+        raise ValueError("device_status must be an int32 device tensor")
+    return device_status.data_ptr()
+
+
+def art_page_summary(k_cache, page_table, seq_lens, summary=None, *, dtype=torch.float32, device_status=None,
+                     stream=None):
+    """Mean key of every referenced page, per kv-head (art_page_summary in
+    art.h).  Returns summary [num_pages, Hkv, d] (float32 or bfloat16)."""
+    _need_cuda(k_cache, page_table, seq_lens, summary)
+    if summary is None:
+        NP, Hkv, _, d = k_cache.shape
+        summary = torch.zeros(NP, Hkv, d, dtype=dtype, device=k_cache.device)
+    ds = [descriptor(t) for t in (k_cache, page_table, seq_lens, summary)]
+    st = _lib.art_page_summary(*[ctypes.byref(x) for x in ds], _status_ptr(device_status), _stream(stream))
+    _check(st, "art_page_summary")
+    return summary
+
+
+def art_build_order_importance(q, summary, page_table, seq_lens, page, *, sm_scale=0.0, block_scores=None,
+                               block_order=None, device_status=None, stream=None):
+    """Importance-first walk order (art_build_order_importance in art.h).
+    Returns (block_order [B, max_blocks] int32, block_scores [B, max_blocks] float32)."""
+    _need_cuda(q, summary, page_table, seq_lens, block_scores, block_order)
+    B, mb = page_table.shape
+    if block_scores is None:
+        block_scores = torch.empty(B, mb, dtype=torch.float32, device=q.device)
+    if block_order is None:
+        block_order = torch.empty(B, mb, dtype=torch.int32, device=q.device)
+    ds = [descriptor(t) for t in (q, summary, page_table, seq_lens, block_scores, block_order)]
+    r = [ctypes.byref(x) for x in ds]
+    st = _lib.art_build_order_importance(*r[:4], int(page), float(sm_scale), r[4], r[5],
+                                         _status_ptr(device_status), _stream(stream))
+    _check(st, "art_build_order_importance")
+    return block_order, block_scores
 
 
 def raw_library():

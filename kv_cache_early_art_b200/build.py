@@ -12,8 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libart.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu",)]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh")] + [
+SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu", "art_order.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh", "art_host.h")] + [
     os.path.join(ROOT, "include", "art.h")]
 
 NVCC_FLAGS = [

@@ -10,6 +10,7 @@
 #include <unordered_map>
 
 #include "../../include/art.h"
+#include "art_host.h"
 #include "art_kernels.cuh"
 
 namespace {
@@ -19,11 +20,9 @@ using art::Layout;
 
 // ---------------------------------------------------------------- checks ----
 
-bool is_null(const art_tensor_t *t) { return t == nullptr || t->data == nullptr; }
-
-int64_t elem_size(int32_t dt) { return dt == ART_BF16 ? 2 : 4; }
-
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+using art_host::aligned;
+using art_host::elem_size;
+using art_host::is_null;
 
 struct Problem {
     int dtype;

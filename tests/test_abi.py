@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("art_decode_attention", "art_decode_attention_ex", "art_build_order_sink_recency",
-              "art_strerror", "art_version"):
+              "art_page_summary", "art_build_order_importance", "art_strerror", "art_version"):
         assert n in names
 
 
@@ -168,3 +168,60 @@ def test_binding_refuses_cpu_tensors(art):
     q = torch.zeros(1, 4, 64)
     with pytest.raises(ValueError):
         art.art_decode_attention(q, q, q, q, q, q, 0.0, 0.0, 0, 0)
+
+
+def _summary_call(art, k, pt, sl, summ, status=None):
+    r = ctypes.byref
+    return art.raw_library().art_page_summary(r(k), r(pt), r(sl), r(summ), status, None)
+
+
+def test_page_summary_errors(art):
+    k, pt, sl, sm = T([10, 2, 64, 128], 1), T([2, 5], 2), T([2], 2), T([10, 2, 128], 0)
+    assert art.raw_library().art_page_summary(None, None, None, None, None, None) == -1
+    k0 = T([10, 2, 64, 128], 1, data=None)
+    assert _summary_call(art, k0, pt, sl, sm) == -1
+    assert _summary_call(art, k, pt, sl, T([10, 2, 64], 0)) == -2          # d mismatch
+    assert _summary_call(art, k, pt, sl, T([9, 2, 128], 0)) == -2          # page count mismatch
+    assert _summary_call(art, k, T([3, 5], 2), sl, sm) == -2               # table rows != B
+    assert _summary_call(art, k, pt, sl, T([10, 2, 128], 2)) == -3         # int summary
+    assert _summary_call(art, k, T([2, 5], 0), sl, sm) == -3               # float page table
+    assert _summary_call(art, T([10, 2, 64, 96], 1), pt, sl, T([10, 2, 96], 0)) == -4
+    assert _summary_call(art, T([10, 2, 64, 128], 1, data=FAKE + 8), pt, sl, sm) == -2
+    assert _summary_call(art, k, pt, sl, T([10, 2, 128], 0, data=FAKE + 4)) == -2
+    assert _summary_call(art, k, pt, sl, sm, status=FAKE + 2) == -2        # misaligned status word
+
+
+def _imp_call(art, q, sm, pt, sl, page, scale, sc, bo):
+    r = ctypes.byref
+    return art.raw_library().art_build_order_importance(r(q), r(sm), r(pt), r(sl), page, scale, r(sc), r(bo),
+                                                        None, None)
+
+
+def test_importance_order_errors(art):
+    q, sm, pt, sl = T([2, 8, 128], 1), T([10, 2, 128], 0), T([2, 5], 2), T([2], 2)
+    sc, bo = T([2, 5], 0), T([2, 5], 2)
+    lib = art.raw_library()
+    assert lib.art_build_order_importance(None, None, None, None, 64, 0.0, None, None, None, None) == -1
+    assert _imp_call(art, q, sm, pt, sl, 64, 0.0, sc, T([2, 5], 2, data=None)) == -1
+    assert _imp_call(art, q, sm, pt, sl, 0, 0.0, sc, bo) == -5                 # page
+    assert _imp_call(art, q, sm, pt, sl, 64, float("nan"), sc, bo) == -5
+    assert _imp_call(art, q, sm, pt, sl, 64, float("inf"), sc, bo) == -5
+    assert _imp_call(art, T([2, 7, 128], 1), sm, pt, sl, 64, 0.0, sc, bo) == -2   # Hq % Hkv
+    assert _imp_call(art, q, T([10, 2, 64], 0), pt, sl, 64, 0.0, sc, bo) == -2    # d mismatch
+    assert _imp_call(art, q, sm, pt, sl, 64, 0.0, T([2, 6], 0), bo) == -2          # scores shape
+    assert _imp_call(art, q, sm, pt, sl, 64, 0.0, sc, T([3, 5], 2)) == -2          # order shape
+    assert _imp_call(art, q, sm, pt, sl, 64, 0.0, T([2, 5], 2), bo) == -3          # int scores
+    assert _imp_call(art, q, sm, pt, sl, 64, 0.0, sc, T([2, 5], 0)) == -3          # float order
+    assert _imp_call(art, T([2, 8, 96], 1), T([10, 2, 96], 0), pt, sl, 64, 0.0, sc, bo) == -4
+    big_q, big_s = T([2, 256, 128], 1), T([10, 256, 128], 0)                       # Hkv * d > 16384
+    assert _imp_call(art, big_q, big_s, pt, sl, 64, 0.0, sc, bo) == -4
+
+
+def test_importance_binding_refuses_cpu_tensors(art):
+    import torch
+    z = torch.zeros(2, 5, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        art.art_page_summary(torch.zeros(10, 2, 64, 128), z, torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        art.art_build_order_importance(torch.zeros(2, 8, 128), torch.zeros(10, 2, 128), z,
+                                       torch.zeros(2, dtype=torch.int32), 64)
