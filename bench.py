@@ -2,9 +2,10 @@
 
 A step is one pass of the whole hot path over one decode batch: one launch
 of the ART walk for every (sequence, kv-head) unit, which builds the default
-walk order (sink block, then newest to oldest) on the fly in its producer.  The K/V cache is
-resident in HBM before timing starts; the L2 is flushed (a 512 MiB write)
-before every step, outside the step's events.
+walk order (sink block, then newest to oldest) on the fly in its producer.
+The K/V cache is resident in HBM before timing starts; the L2 is flushed before every step,
+outside the step's events (a 512 MiB write, then a 512 MiB read so that the
+flush's dirty lines are not written back inside the step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-cpu-baseline] [--no-e2e]
@@ -40,6 +41,24 @@ WORKLOAD_TEXT = {
 }
 SPEC_HBM_GBS = 8000.0
 L2_FLUSH_BYTES = 512 << 20
+
+
+class L2Flush:
+    """Evicts the K/V cache from L2 before a step, outside its events: a write
+    of a 512 MiB buffer (4x the 126 MB L2), then a read of a second one, so
+    that the step starts with L2 holding only clean lines of an unrelated
+    buffer.  Without the read the write's dirty lines would be written back
+    to HBM during the step and counted against it."""
+
+    def __init__(self, torch, dev):
+        self.torch = torch
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.int64, device=dev)
+
+    def __call__(self, i):
+        self.w.fill_(i)
+        self.torch.sum(self.r, dim=0, dtype=self.torch.int64, out=self.acc)
 
 
 def measured_peaks():
@@ -234,7 +253,8 @@ def config_for(name, w, gpus):
            "params": ({"eps_m": p[0], "eps_d": p[1], "P": int(p[2]), "min_blocks": int(p[3])} if p else
                       "per-sequence"),
            "order": "sink block, then newest to oldest (built on the fly inside the walk)",
-           "l2": "flushed before every step (512 MiB write, outside the step events)",
+           "l2": "flushed before every step, outside the step events: 512 MiB write, then a 512 MiB read "
+                 "so that no dirty line of the flush is written back inside the step",
            "parallelism": f"replicas x{gpus} (independent batches, no collective)"}
     return cfg
 
@@ -267,7 +287,7 @@ def run_ours(args):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     out = torch.empty(B, w.Hq, d, dtype=torch.float32, device=dev)
     stop = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(torch, dev)
 
     def step(eps_off=False):
         kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
@@ -281,7 +301,7 @@ def run_ours(args):
         Returns per-step ms (twice: the whole step is the walk)."""
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
         for i in range(n):
-            flush.fill_(i)
+            flush(i)
             ev[i][0].record(stream)
             kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                       P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
@@ -377,7 +397,7 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         e_ms = []
         for i in range(args.steps):
-            flush.fill_(i)
+            flush(i)
             a = torch.cuda.Event(enable_timing=True)
             b_ = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -417,7 +437,7 @@ def run_table(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(torch, dev)
     peak, _ = measured_peaks()
     inf = float("inf")
     rows = []
@@ -425,7 +445,7 @@ def run_table(args):
     def median_ms(fn):
         ts = []
         for i in range(args.table_reps):
-            flush.fill_(i)
+            flush(i)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
