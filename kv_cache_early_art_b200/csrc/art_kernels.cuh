@@ -534,7 +534,8 @@ struct CudaEngine {
 #pragma unroll
         for (int bt = 0; bt < NB; ++bt) {
             const int t = bt * TB + lane / GMAX;
-            const float p = (sc[bt] == -CUDART_INF_F) ? 0.f : exp2f(sc[bt] - m);
+            // ex2.approx: relative error below 2^-22, far inside the fp32 tolerance
+            const float p = (sc[bt] == -CUDART_INF_F) ? 0.f : ex2_approx(sc[bt] - m);
             l += p;
             if (t < PAGE)
                 pbuf[t * GMAX + gl] = p;
@@ -583,7 +584,7 @@ struct CudaEngine {
         for (int g = 0; g < GMAX; ++g) {
             const float lg = __shfl_sync(0xffffffffu, l, g);
             if (g < a.G) {
-                const float inv = lg > 0.f ? 1.f / lg : 0.f;
+                const float inv = lg > 0.f ? rcp_approx(lg) : 0.f;
                 const uint32_t addr = sr.base + 4u * (u_off + g * D + lane * DE);
                 if constexpr (DE == 4)
                     st_async_v4(addr, acc[g][0] * inv, acc[g][1] * inv, acc[g][2] * inv, acc[g][3] * inv,
@@ -632,14 +633,17 @@ struct MmaEngine {
 
         // scores, rows = tokens, columns = heads
         // (even and odd head-dim steps accumulate separately: shorter mma chains)
+        // (head-dim steps outer, token tiles inner: 2*MT independent mma chains)
         float sacc[MT][4], sodd[MT][4];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 sacc[mt][i] = sodd[mt][i] = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
+        for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
                 const int t = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int d = ks * 16 + (lane >> 4) * 8;
                 uint32_t a0, a1, a2, a3;
@@ -647,18 +651,24 @@ struct MmaEngine {
                 mma_bf16_16816((ks & 1) ? sodd[mt] : sacc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
             }
 #pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
             for (int i = 0; i < 4; ++i)
                 sacc[mt][i] += sodd[mt][i];
-        }
+        // The max is taken on the raw scores (the scale is positive, so it
+        // commutes with the max, bit for bit); each weight is then one fma and
+        // one ex2.approx (relative error below 2^-22, far inside the ~16 bits
+        // the bf16 hi + lo split of P keeps).
         const int g0 = 2 * c;
+        const bool hv0 = g0 < a.G, hv1 = g0 + 1 < a.G;
         float m2[2] = {-CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = mt * 16 + r + (i >> 1) * 8;
-                const bool valid = (t < nv) && (g0 + (i & 1) < a.G);
-                sacc[mt][i] = valid ? sacc[mt][i] * a.scale_log2 : -CUDART_INF_F;
+                const bool valid = (t < nv) && ((i & 1) ? hv1 : hv0);
+                sacc[mt][i] = valid ? sacc[mt][i] : -CUDART_INF_F;
                 m2[i & 1] = fmaxf(m2[i & 1], sacc[mt][i]);
             }
 #pragma unroll
@@ -666,12 +676,15 @@ struct MmaEngine {
             m2[0] = fmaxf(m2[0], __shfl_xor_sync(0xffffffffu, m2[0], off));
             m2[1] = fmaxf(m2[1], __shfl_xor_sync(0xffffffffu, m2[1], off));
         }
+        m2[0] *= a.scale_log2;
+        m2[1] *= a.scale_log2;
         float l2[2] = {0.f, 0.f};
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float p = (sacc[mt][i] == -CUDART_INF_F) ? 0.f : exp2f(sacc[mt][i] - m2[i & 1]);
+                const float sv = sacc[mt][i];
+                const float p = (sv == -CUDART_INF_F) ? 0.f : ex2_approx(fmaf(sv, a.scale_log2, -m2[i & 1]));
                 sacc[mt][i] = p;
                 l2[i & 1] += p;
             }
@@ -716,14 +729,17 @@ struct MmaEngine {
             fence_proxy_async_smem();
             __syncwarp();
         }
+        // (token steps outer, head-dim tiles inner: KS independent mma chains)
         float oacc[KS][4], oacc2[KS][4];
 #pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
+        for (int dt = 0; dt < KS; ++dt)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 oacc[dt][i] = oacc2[dt][i] = 0.f;
 #pragma unroll
-            for (int kt2 = 0; kt2 < MT; ++kt2) {
+        for (int kt2 = 0; kt2 < MT; ++kt2)
+#pragma unroll
+            for (int dt = 0; dt < KS; ++dt) {
                 const int t = kt2 * 16 + (lane & 7) + (lane >> 4) * 8;
                 const int d = dt * 16 + ((lane >> 3) & 1) * 8;
                 uint32_t a0, a1, a2, a3;
@@ -732,7 +748,6 @@ struct MmaEngine {
                 if constexpr (!kShared)
                     mma_bf16_16816(oacc2[dt], a0, a1, a2, a3, bl[kt2][0], bl[kt2][1]);
             }
-        }
         __syncwarp();
         if (lane == 0)
             mbar_arrive(sh.empty(s, a.S));
@@ -758,8 +773,8 @@ struct MmaEngine {
         }
         if (writer) {
             const bool w0 = gA < a.G, w1 = gA + 1 < a.G;
-            const float inv0 = (w0 && l2[0] > 0.f) ? 1.f / l2[0] : 0.f;
-            const float inv1 = (w1 && l2[1] > 0.f) ? 1.f / l2[1] : 0.f;
+            const float inv0 = (w0 && l2[0] > 0.f) ? rcp_approx(l2[0]) : 0.f;
+            const float inv1 = (w1 && l2[1] > 0.f) ? rcp_approx(l2[1]) : 0.f;
             if (r == 0) {
                 if (w0) {
                     st_async_b32(sr.base + 4u * (4 + gA), __float_as_uint(m2[0]), sr.ready);
