@@ -260,7 +260,7 @@ struct Shared {
 
 template <typename T, int D, int PAGE, int ENGINE>
 __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUtensorMap *tmk, const CUtensorMap *tmv,
-                              int b, int h, int N, int Lseq, uint32_t rank)
+                              int b, int h, int N, int Lseq, uint32_t rank, int first_lb, int first_pp)
 {
     const int lane = threadIdx.x & 31;
     const int S = a.S, R = a.R, C = a.C;
@@ -275,7 +275,8 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
     uint32_t kphase = 0, vphase = 0;  // bit s: parity of the last phase armed on full_k[s] / full_v[s]
     uint32_t kused = 0, vused = 0;
     uint32_t touched = 0;        // this CTA's walk steps whose page was read (loaded or prefetched)
-    int batch_k0 = -1, my_lb = -1, my_pp = -1;
+    // the first 32 index pairs were loaded before the set-up barriers
+    int batch_k0 = 0, my_lb = first_lb, my_pp = first_pp;
     // L2 prefetch front: step k + PFS, PFS = ceil(PF / C) of this CTA's steps
     const int PFS = (a.PF + C - 1) / C;
     int pbatch_k0 = -1, my_plb = -1, my_ppp = -1;
@@ -797,13 +798,15 @@ struct MmaEngine {
 };
 
 template <typename T, int D, int PAGE, int GMAX, int ENGINE>
-__device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h, int cw)
+using EngineFor = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX>,
+                                            CudaEngine<T, D, PAGE, GMAX>>::type;
+
+// eng holds the unit's queries, loaded before the set-up barriers
+template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+__device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h, int cw,
+                             EngineFor<T, D, PAGE, GMAX, ENGINE> &eng)
 {
     const int lane = threadIdx.x & 31;
-    using Engine = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX>,
-                                             CudaEngine<T, D, PAGE, GMAX>>::type;
-    Engine eng;
-    eng.load_q(a, b, h, lane);
     float *pbuf = sh.pbuf + (ENGINE == kEngineMma ? 0 : cw * PAGE * GMAX);
     const uint32_t ring_cl = mapa(smem_u32(sh.ring), 0);
     const uint32_t ready_cl = mapa(sh.ready(0, a.S), 0);
@@ -1248,6 +1251,23 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int N = Lseq <= 0 ? 0 : (Lseq + PAGE - 1) / PAGE;
     const bool bad_len = N > a.max_blocks;
 
+    constexpr int NM = MergeShape<D, GMAX, ENGINE, NMW>::NM;
+    const bool walk = N > 0 && !bad_len;
+    const int lane = threadIdx.x & 31;
+    // Start the first global reads now, so that they are in flight during the
+    // set-up barriers: the producer's first 32 (block, page) pairs, the compute
+    // warps' queries.
+    int first_lb = -1, first_pp = -1;
+    if (walk && warp == 0) {
+        const int jj = (int)rank + lane * a.C;
+        if (jj < N)
+            // no order given: the sink block, then newest to oldest
+            first_lb = a.block_order ? __ldg(a.block_order + (int64_t)b * a.bo_sb + jj) : (jj == 0 ? 0 : N - jj);
+    }
+    EngineFor<T, D, PAGE, GMAX, ENGINE> eng;
+    if (walk && warp > NM)
+        eng.load_q(a, b, h, lane);
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.S; ++s) {
             mbar_init(sh.full_k(s), 1);
@@ -1263,19 +1283,19 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         fence_mbar_init_cluster();
     }
     __syncthreads();
+    if (walk && warp == 0 && first_lb >= 0 && first_lb < N)
+        first_pp = __ldg(a.page_table + (int64_t)b * a.pt_sb + first_lb);
     cluster_sync();  // remote CTAs may now arrive on the leader's barriers
 
-    constexpr int NM = MergeShape<D, GMAX, ENGINE, NMW>::NM;
-    if (N > 0 && !bad_len) {
+    if (walk) {
         if (warp == 0)
-            producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank);
+            producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank, first_lb, first_pp);
         else if (warp <= NM) {
             if (rank == 0)
                 merge_role<D, GMAX, ENGINE, NMW>(a, sh, b, h, N, warp - 1);
         } else
-            compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM);
+            compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM, eng);
     } else if (rank == 0 && warp == 1) {
-        const int lane = threadIdx.x & 31;
         float *op = a.out + (int64_t)b * a.out_sb;
         for (int i = lane; i < a.G * D; i += 32)
             op[(int64_t)(h * a.G + i / D) * a.out_sh + i % D] = 0.f;
