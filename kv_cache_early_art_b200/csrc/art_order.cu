@@ -242,13 +242,14 @@ __global__ void __launch_bounds__(kThreads) art_block_score_kernel(ScoreArgs a)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int L = a.sl[b];
-    const int N = min(n_blocks_of(L, a.page), a.max_blocks);
     const int NBW = a.blocks_per_warp;                // even, at most 32
     const int jw = (blockIdx.x * kWarps + warp) * NBW;
-    // this warp's page indices, one coalesced load, in flight during the prologue
+    // The sequence length, this warp's page indices (read up to the table's
+    // width; entries past the sequence are ignored below) and the query rows
+    // are independent reads: all of them go out before any is waited for.
+    const int L = a.sl[b];
     int pidx = -1;
-    if (lane < NBW && jw + lane < N)
+    if (lane < NBW && jw + lane < a.max_blocks)
         pidx = a.pt[(int64_t)b * a.pts0 + jw + lane];
     const int HD = a.Hkv * a.d;
     const TQ *qb = static_cast<const TQ *>(a.q) + (int64_t)b * a.qs0;
@@ -269,6 +270,9 @@ __global__ void __launch_bounds__(kThreads) art_block_score_kernel(ScoreArgs a)
         *reinterpret_cast<float4 *>(qg + idx) = make_float4(s[0], s[1], s[2], s[3]);
     }
     __syncthreads();
+    const int N = min(n_blocks_of(L, a.page), a.max_blocks);
+    if (jw + lane >= N)
+        pidx = -1;
     if (blockIdx.x == 0 && threadIdx.x == 0 && n_blocks_of(L, a.page) > a.max_blocks)
         report(a.status, ART_ERR_BAD_INDEX);
     const int VR = a.d / VE;
