@@ -1253,20 +1253,19 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
     constexpr int NM = MergeShape<D, GMAX, ENGINE, NMW>::NM;
     const bool walk = N > 0 && !bad_len;
-    const int lane = threadIdx.x & 31;
     // Start the first global reads now, so that they are in flight during the
     // set-up barriers: the producer's first 32 (block, page) pairs, the compute
     // warps' queries.
     int first_lb = -1, first_pp = -1;
     if (walk && warp == 0) {
-        const int jj = (int)rank + lane * a.C;
+        const int jj = (int)rank + (threadIdx.x & 31) * a.C;
         if (jj < N)
             // no order given: the sink block, then newest to oldest
             first_lb = a.block_order ? __ldg(a.block_order + (int64_t)b * a.bo_sb + jj) : (jj == 0 ? 0 : N - jj);
     }
     EngineFor<T, D, PAGE, GMAX, ENGINE> eng;
     if (walk && warp > NM)
-        eng.load_q(a, b, h, lane);
+        eng.load_q(a, b, h, threadIdx.x & 31);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.S; ++s) {
@@ -1296,6 +1295,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         } else
             compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM, eng);
     } else if (rank == 0 && warp == 1) {
+        const int lane = threadIdx.x & 31;
         float *op = a.out + (int64_t)b * a.out_sb;
         for (int i = lane; i < a.G * D; i += 32)
             op[(int64_t)(h * a.G + i / D) * a.out_sh + i % D] = 0.f;
