@@ -297,7 +297,8 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
     // with fewer units each unit is split over a cluster and needs a deeper
     // window to cover the latency from fetch to merged stop decision.
     static const int many_units[][3] = {{2, 2, 16}, {1, 2, 16}, {2, 2, 8}, {1, 2, 8}};
-    static const int few_units_large[][3] = {{4, 4, 24}, {2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
+    static const int few_units_large[][3] = {{5, 5, 28}, {4, 4, 24}, {2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16},
+                                             {1, 2, 8}};
     static const int few_units_small[][3] = {{4, 8, 32}, {4, 8, 16}, {4, 4, 16}, {2, 4, 16}, {2, 2, 8},
                                              {1, 2, 8}};
     const int(*cand)[3];
@@ -307,7 +308,7 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         ncand = 4;
     } else if (tile >= 16384) {
         cand = few_units_large;
-        ncand = 6;
+        ncand = 7;
     } else {
         cand = few_units_small;
         ncand = 6;
@@ -344,10 +345,8 @@ art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const Device
         return ART_ERR_LAUNCH;
     per_sm = per_sm < 1 ? 1 : per_sm;
     const int slots = di.sms * per_sm;
-    int C = slots / units;
-    C = C < 1 ? 1 : (C > 16 ? 16 : C);
-    // the largest cluster size whose clusters all fit at once
-    for (; C > 1; --C) {
+    // clusters of C CTAs that can be resident at once (0 if none)
+    auto resident = [&](int C) -> int {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -360,9 +359,37 @@ art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const Device
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, (void *)fn, &cfg) == cudaSuccess && nclusters >= units)
-            break;
-        cudaGetLastError();
+        if (cudaOccupancyMaxActiveClusters(&nclusters, (void *)fn, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        return nclusters;
+    };
+    int C = 1;
+    if (units < slots) {
+        // one wave: the largest cluster size whose clusters all fit at once
+        C = slots / units;
+        C = C > 16 ? 16 : C;
+        for (; C > 1; --C)
+            if (resident(C) >= units)
+                break;
+    } else {
+        // several waves of units: a unit split over C CTAs takes about 1/C of
+        // the time, and the launch takes ceil(units / resident clusters)
+        // rounds, so pick the C with the fewest rounds / C (the smaller C on
+        // a tie: it has no cross-CTA merge traffic)
+        long best_num = (units + slots - 1) / slots, best_den = 1;   // C = 1
+        for (int c = 2; c <= 4; c *= 2) {
+            const int rc = resident(c);
+            if (rc <= 0)
+                continue;
+            const long rounds = (units + rc - 1) / rc;
+            if (rounds * best_den < best_num * c) {
+                best_num = rounds;
+                best_den = c;
+                C = c;
+            }
+        }
     }
     s->C = C;
     (void)ka;

@@ -238,3 +238,44 @@ def test_qwen7b_b4_full_size(cuda_lib):
 
 def test_mistral7b_b128_full_size(cuda_lib):
     _full(cuda_lib, "mistral7b_b128", list(range(0, 128, 9)))
+
+
+SHAPES = {
+    # (cluster, compute warps, stages, window): every (warps, stages) pairing
+    # the launch accepts, from the smallest ring to the deepest window
+    "bf16": [(1, 1, 2, 8), (2, 2, 2, 16), (2, 3, 3, 24), (2, 4, 4, 24), (2, 5, 5, 28), (3, 2, 4, 16),
+             (4, 1, 2, 8), (2, 2, 4, 32)],
+    "f32": [(1, 1, 2, 8), (2, 5, 5, 28), (2, 6, 6, 16), (2, 3, 6, 16), (3, 2, 4, 24), (2, 4, 8, 16)],
+}
+
+
+@pytest.mark.parametrize("dtype,engine", [("bf16", 2), ("bf16", 1), ("f32", 1)])
+def test_launch_shapes(cuda_lib, dtype, engine):
+    """Explicit launch shapes: the stop and the output do not depend on how
+    the walk is spread over CTAs, warps, stages and the window (block states
+    are exact per block and the merge folds fixed batches in walk order), so
+    every shape equals the library's own choice bit for bit, and that one
+    matches the oracle."""
+    page = 64 if dtype == "bf16" else 16
+    w = make_custom(B=4, Hq=12, Hkv=3, d=128, page=page, dtype=dtype,
+                    seq_lens=[page * 90 + 7, page * 40, 1, page * 130 + page // 2], seed=31, planted=3,
+                    planted_gain=5.0, order="random", eps_m=5e-3, eps_d=5e-4, P=[2, 1, 3, 2],
+                    min_blocks=[1, 2, 1, 4])
+    out0, stop0, fetched0, status, info0 = run_gpu(cuda_lib, w, engine=engine)
+    assert status == 0
+    parity.check(w, out0, stop0)
+    ran = 0
+    for (cl, nw, st, win) in SHAPES[dtype]:
+        try:
+            out, stop, fetched, status, info = run_gpu(cuda_lib, w, engine=engine, cluster_size=cl,
+                                                       compute_warps=nw, stages=st, window=win)
+        except cuda_lib.ArtError as e:
+            assert "UNSUPPORTED" in str(e), e     # this shape's ring does not fit in shared memory
+            continue
+        ran += 1
+        assert status == 0
+        assert (info["cluster_size"], info["compute_warps"], info["stages"], info["window"]) == (cl, nw, st, win)
+        assert torch.equal(stop, stop0), (cl, nw, st, win)
+        assert torch.equal(out, out0), (cl, nw, st, win)
+        assert_fetch_bound(w, stop, fetched, win + info["prefetch"])
+    assert ran >= len(SHAPES[dtype]) - 1
