@@ -297,8 +297,8 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
     // with fewer units each unit is split over a cluster and needs a deeper
     // window to cover the latency from fetch to merged stop decision.
     static const int many_units[][3] = {{2, 2, 16}, {1, 2, 16}, {2, 2, 8}, {1, 2, 8}};
-    static const int few_units_large[][3] = {{5, 5, 28}, {4, 4, 24}, {2, 4, 24}, {2, 4, 16}, {2, 2, 16}, {1, 2, 16},
-                                             {1, 2, 8}};
+    static const int few_units_large[][3] = {{5, 5, 28}, {4, 4, 24}, {2, 4, 24}, {3, 3, 24}, {2, 2, 24},
+                                             {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
     static const int few_units_small[][3] = {{4, 8, 32}, {4, 8, 16}, {4, 4, 16}, {2, 4, 16}, {2, 2, 8},
                                              {1, 2, 8}};
     const int(*cand)[3];
@@ -308,7 +308,7 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         ncand = 4;
     } else if (tile >= 16384) {
         cand = few_units_large;
-        ncand = 7;
+        ncand = 9;
     } else {
         cand = few_units_small;
         ncand = 6;

@@ -876,8 +876,11 @@ struct MergeShape {
     static constexpr int NM0 = NMW > NMIN ? NMW : NMIN;
     static constexpr int NM = NM0 < Lay::NV ? NM0 : Lay::NV;
     static constexpr int NVW = Lay::NV / NM;
-    static constexpr int KB = (32 / GMAX) < 8 ? (32 / GMAX) : 8;
+    static constexpr int KB = 8;                  // blocks per merge batch
+    static constexpr int KH = 32 / GMAX;          // blocks per row of scan lanes
+    static constexpr int NH = KB > KH ? KB / KH : 1;  // (block, head) entries per scan lane
     static_assert(Lay::NV % NM == 0, "merge split");
+    static_assert(NH * KH >= KB && NH <= 2, "scan rows");
 };
 
 __device__ __forceinline__ void merge_barrier(int nthreads)
@@ -905,7 +908,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 {
     using MS = MergeShape<D, GMAX, ENGINE, NMW>;
     using Lay = typename MS::Lay;
-    constexpr int NVW = MS::NVW, VW = Lay::VW, VP = VW / 2, KB = MS::KB, NM = MS::NM;
+    constexpr int NVW = MS::NVW, VW = Lay::VW, VP = VW / 2, KB = MS::KB, NM = MS::NM, KH = MS::KH, NH = MS::NH;
     static_assert(KB <= 8, "two partial sums per block in 16 lanes");
     const int lane = threadIdx.x & 31;
     const int G = a.G;
@@ -918,8 +921,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     const int slot_floats = (int)(sh.L.slot_bytes / 4);
     const int vbase = mw * NVW;
 
-    // scan lane: block kl of the batch, head gl; it also keeps the running
-    // softmax scalars of head gl
+    // scan lane: blocks kl (and kl + KH) of the batch, head gl; it also keeps
+    // the running softmax scalars of head gl
     const int kl = lane / GMAX, gl = lane % GMAX;
     float Mx = -CUDART_INF_F, Lm = 0.f;
     // running output of this lane's elements, as packed fp32 pairs
@@ -956,17 +959,18 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     // o += Delta; with sums, add o.Delta and |Delta|^2 of the slice to pd, pe.
     auto fold = [&](int k, float beta, const uint64_t (&uv)[NVW][VP], float &pd, float &pe, bool sums) {
         uint64_t bp[NVW];
+        const int kr = NH > 1 ? k % KH : k;  // row of the scan lanes holding block k
         if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads
             const int h0 = Lay::head(lane, 0, 0);
-            const float b0 = __shfl_sync(0xffffffffu, beta, k * GMAX + h0);
-            const float b1 = __shfl_sync(0xffffffffu, beta, k * GMAX + h0 + 1);
+            const float b0 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0);
+            const float b1 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0 + 1);
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii)
                 bp[ii] = pk2(b0, b1);
         } else {  // vector i holds head i
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii) {
-                const float bi = __shfl_sync(0xffffffffu, beta, k * GMAX + vbase + ii);
+                const float bi = __shfl_sync(0xffffffffu, beta, kr * GMAX + vbase + ii);
                 bp[ii] = (vbase + ii < G) ? pk2(bi, bi) : 0ull;
             }
         }
@@ -988,7 +992,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         }
     };
     // fold blocks 0..kend of the batch starting at slot s0 (u loads one block ahead)
-    auto fold_batch = [&](int s0, int kend, float beta, float (&v)[16], bool sums) {
+    auto fold_batch = [&](int s0, int kend, float beta, float beta_hi, float (&v)[16], bool sums) {
         uint64_t ua[NVW][VP], ub[NVW][VP];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
 #pragma unroll
@@ -1000,7 +1004,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            fold(k, beta, (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
+            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
         }
     };
 
@@ -1071,33 +1075,83 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 #pragma unroll
         for (int q = 0; q < 16; ++q)
             v[q] = 0.f;
-        float beta = 0.f, n0part = 0.f;
+        float beta = 0.f, beta_hi = 0.f, n0part = 0.f;  // beta_hi: blocks KH.. (two scan rows)
         uint64_t o0[NVW][VP];
         if (!local_fail) {
             // 2. shares of the softmax mass: beta_(k,g) = w_k / (L_prev + w_0 + ... + w_k)
-            float mk = -CUDART_INF_F, lk = 0.f;
-            if (kl < nb && gl < G) {
-                int sl = s0 + kl;
-                sl = sl >= a.R ? sl - a.R : sl;
-                const float *sp = sh.ring + (size_t)sl * slot_floats;
-                mk = sp[4 + gl];
-                lk = sp[4 + GMAX + gl];
-            }
-            float Mb = fmaxf(Mx, mk);
+            float Mb;
+            if constexpr (NH == 1) {  // one (block, head) entry per lane
+                float mk = -CUDART_INF_F, lk = 0.f;
+                if (kl < nb && gl < G) {
+                    int sl = s0 + kl;
+                    sl = sl >= a.R ? sl - a.R : sl;
+                    const float *sp = sh.ring + (size_t)sl * slot_floats;
+                    mk = sp[4 + gl];
+                    lk = sp[4 + GMAX + gl];
+                }
+                Mb = fmaxf(Mx, mk);
 #pragma unroll
-            for (int off = GMAX; off < 32; off <<= 1)
-                Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
-            const float w = (mk == -CUDART_INF_F) ? 0.f : lk * ex2_approx(mk - Mb);
-            float S = w;
+                for (int off = GMAX; off < 32; off <<= 1)
+                    Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
+                const float w = (mk == -CUDART_INF_F) ? 0.f : lk * ex2_approx(mk - Mb);
+                float S = w;
 #pragma unroll
-            for (int off = GMAX; off < 32; off <<= 1) {
-                const float t = __shfl_up_sync(0xffffffffu, S, off);
-                if (lane >= off)
-                    S += t;
+                for (int off = GMAX; off < 32; off <<= 1) {
+                    const float t = __shfl_up_sync(0xffffffffu, S, off);
+                    if (lane >= off)
+                        S += t;
+                }
+                const float Lam = ((Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb)) + S;
+                beta = Lam > 0.f ? w * rcp_approx(Lam) : 0.f;
+                Lm = __shfl_sync(0xffffffffu, Lam, (nb - 1) * GMAX + gl);
+            } else {  // two rows: entry hh of a lane is block kl + hh KH
+                float mk[NH], lk[NH];
+                Mb = Mx;
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh) {
+                    const int k = kl + hh * KH;
+                    mk[hh] = -CUDART_INF_F;
+                    lk[hh] = 0.f;
+                    if (k < nb && gl < G) {
+                        int sl = s0 + k;
+                        sl = sl >= a.R ? sl - a.R : sl;
+                        const float *sp = sh.ring + (size_t)sl * slot_floats;
+                        mk[hh] = sp[4 + gl];
+                        lk[hh] = sp[4 + GMAX + gl];
+                    }
+                    Mb = fmaxf(Mb, mk[hh]);
+                }
+#pragma unroll
+                for (int off = GMAX; off < 32; off <<= 1)
+                    Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
+                float w[NH], S[NH];
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh) {
+                    w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : lk[hh] * ex2_approx(mk[hh] - Mb);
+                    S[hh] = w[hh];
+                }
+#pragma unroll
+                for (int off = GMAX; off < 32; off <<= 1)
+#pragma unroll
+                    for (int hh = 0; hh < NH; ++hh) {
+                        const float t = __shfl_up_sync(0xffffffffu, S[hh], off);
+                        if (lane >= off)
+                            S[hh] += t;
+                    }
+                if constexpr (NH > 1)  // the second row follows the whole first row
+                    S[1] += __shfl_sync(0xffffffffu, S[0], (KH - 1) * GMAX + gl);
+                const float base = (Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb);
+                float Lam[NH], bh[NH];
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh) {
+                    Lam[hh] = base + S[hh];
+                    bh[hh] = Lam[hh] > 0.f ? w[hh] * rcp_approx(Lam[hh]) : 0.f;
+                }
+                beta = bh[0];
+                beta_hi = bh[NH - 1];
+                const float Llast = (NH > 1 && nb - 1 >= KH) ? Lam[NH - 1] : Lam[0];
+                Lm = __shfl_sync(0xffffffffu, Llast, ((nb - 1) % KH) * GMAX + gl);
             }
-            const float Lam = ((Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb)) + S;
-            beta = Lam > 0.f ? w * rcp_approx(Lam) : 0.f;
-            Lm = __shfl_sync(0xffffffffu, Lam, (nb - 1) * GMAX + gl);
             Mx = Mb;
             // 3. ||o||^2 before the batch, then fold the batch into this warp's slice
             uint64_t n2 = 0ull;
@@ -1109,7 +1163,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                     n2 = fma2(o[i][q], o[i][q], n2);
                 }
             n0part = lo2(n2) + hi2(n2);
-            fold_batch(s0, nb - 1, beta, v, true);
+            fold_batch(s0, nb - 1, beta, beta_hi, v, true);
         }
         // 4. lane 2k+q (and 2k+q+16): sum over the warp of quantity q of batch block k
         reduce_scatter16(v, lane);
@@ -1186,7 +1240,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 #pragma unroll
                     for (int q = 0; q < VP; ++q)
                         o[i][q] = o0[i][q];
-                fold_batch(s0, kstop, beta, v, false);
+                fold_batch(s0, kstop, beta, beta_hi, v, false);
             }
         }
         // Slots of this batch are free again (or the walk is over).  Every value
