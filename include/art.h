@@ -152,6 +152,37 @@ typedef struct {
 art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream);
 
 /*
+ * art_decode_attention_multi -- n_queries query tokens of each sequence (for
+ * example draft tokens being verified together) share one walk of its cache:
+ * every block is fetched once for all of them.  This is the decode form of
+ * the cross-query reuse of shared KV entries in "QUILT: Rethinking
+ * Sparse-Attention Prefill through Shared Query Execution" (Abstract); the
+ * ART pages themselves only walk one query.
+ *
+ * Result: token t of sequence b gets exactly what art_decode_attention_ex
+ * gives for q[b, t] alone -- its own statistics over its Hq/Hkv heads, its
+ * own patience counter and stop, its output at its own stop.  The walk of a
+ * (sequence, kv-head) ends when every token has stopped, so the blocks read
+ * are those up to the latest token's stop, instead of each token reading its
+ * own prefix.  All tokens of a sequence use the same order, page table,
+ * thresholds and min_blocks.
+ *
+ * Tensors in p (everything else as in art_decode_attention_ex):
+ *  q           [B, n_queries, Hq, d]   F32 or BF16; d contiguous; the token and
+ *                                      head strides multiples of 16 bytes.
+ *  out         [B, n_queries, Hq, d]   F32.
+ *  stop_block  [B, n_queries, Hkv]     I32: blocks consumed by each token.
+ * p->blocks_fetched counts the pages read by the shared walk of each unit.
+ * Supported: n_queries = 1 (the single-query walk, on [B, 1, ...] tensors;
+ * any size art_decode_attention_ex takes) or 2; with 2, d = 128 and
+ * 2 * Hq/Hkv <= 8 (both tokens' heads fit the eight rows of one unit); BF16
+ * on the tensor-core engine (engine 0 or 2), F32 on the CUDA-core engine.
+ * Other cases return ART_ERR_UNSUPPORTED.
+ * Errors as in art_decode_attention_ex; the library allocates nothing.
+ */
+art_status_t art_decode_attention_multi(const art_params_t *p, int32_t n_queries, art_stream_t stream);
+
+/*
  * art_build_order_sink_recency -- write the default walk order: for each
  * sequence b with N_b = ceil(seq_lens[b] / page) blocks, block_order[b] =
  * [0, N_b-1, N_b-2, ..., 1] followed by -1 up to max_blocks (the sink block

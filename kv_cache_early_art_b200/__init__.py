@@ -9,7 +9,8 @@ calling any attention entry point without the library raises ImportError.
 from importlib import import_module
 
 _BINDING_NAMES = {
-    "art_decode_attention", "art_decode_attention_ex", "art_build_order_sink_recency", "art_strerror",
+    "art_decode_attention", "art_decode_attention_ex", "art_decode_attention_multi",
+    "art_build_order_sink_recency", "art_strerror",
     "art_page_summary", "art_build_order_importance",
     "art_version", "ArtError", "descriptor", "raw_library", "ENGINE_AUTO", "ENGINE_CUDA", "ENGINE_MMA",
     "STATUS", "ArtParams", "ArtTensor", "ArtLaunchInfo", "LIB_PATH",

@@ -66,6 +66,8 @@ _lib.art_decode_attention.argtypes = [_P(ArtTensor)] * 6 + [ctypes.c_float, ctyp
 _lib.art_decode_attention.restype = ctypes.c_int
 _lib.art_decode_attention_ex.argtypes = [_P(ArtParams), ctypes.c_void_p]
 _lib.art_decode_attention_ex.restype = ctypes.c_int
+_lib.art_decode_attention_multi.argtypes = [_P(ArtParams), ctypes.c_int32, ctypes.c_void_p]
+_lib.art_decode_attention_multi.restype = ctypes.c_int
 _lib.art_build_order_sink_recency.argtypes = [_P(ArtTensor), ctypes.c_int32, _P(ArtTensor), ctypes.c_void_p]
 _lib.art_build_order_sink_recency.restype = ctypes.c_int
 _lib.art_page_summary.argtypes = [_P(ArtTensor)] * 4 + [ctypes.c_void_p, ctypes.c_void_p]
@@ -142,24 +144,15 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
     return out, stop_block
 
 
-def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_lens, *, eps_m=0.0, eps_d=0.0,
-                            P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
-                            P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
-                            engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                            debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None, want_info=False):
-    """art_decode_attention_ex in art.h.  Per-sequence arrays are device
-    tensors of length B (float32 thresholds, int32 P / min_blocks).
-    Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
+def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P, min_blocks,
+            sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status,
+            engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch):
+    """Fill art_params_t (argument marshalling only); returns (params, info)."""
     per = [eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status]
     _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, *per)
     for t, dt in zip(per, (torch.float32, torch.float32, torch.int32, torch.int32, torch.int32, torch.int32)):
         if t is not None and (t.dtype != dt or not t.is_contiguous()):
             raise ValueError(f"per-sequence/accounting arrays must be contiguous {dt}")
-    B, Hq, d = q.shape
-    if out is None:
-        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
-    if stop_block is None:
-        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
     p = ArtParams()
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("page_table", page_table),
                     ("block_order", block_order), ("seq_lens", seq_lens), ("out", out), ("stop_block", stop_block)):
@@ -179,8 +172,53 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p.prefetch = int(prefetch)
     info = ArtLaunchInfo()
     p.info = ctypes.pointer(info)
+    return p, info
+
+
+def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_lens, *, eps_m=0.0, eps_d=0.0,
+                            P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
+                            P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
+                            engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
+                            debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None, want_info=False):
+    """art_decode_attention_ex in art.h.  Per-sequence arrays are device
+    tensors of length B (float32 thresholds, int32 P / min_blocks).
+    Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
+                      min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
+                      blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
+                      timeout_ns, debug_flags, prefetch)
     st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
     _check(st, "art_decode_attention_ex")
+    if want_info:
+        return out, stop_block, info.as_dict()
+    return out, stop_block
+
+
+def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq_lens, *, eps_m=0.0, eps_d=0.0,
+                               P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
+                               P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
+                               engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
+                               debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None,
+                               want_info=False):
+    """art_decode_attention_multi in art.h: q [B, T, Hq, d], T query tokens
+    per sequence sharing one walk.  Returns (out [B, T, Hq, d],
+    stop_block [B, T, Hkv]) or those plus the launch info dict."""
+    B, T, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, T, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, T, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
+                      min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
+                      blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
+                      timeout_ns, debug_flags, prefetch)
+    st = _lib.art_decode_attention_multi(ctypes.byref(p), int(T), _stream(stream))
+    _check(st, "art_decode_attention_multi")
     if want_info:
         return out, stop_block, info.as_dict()
     return out, stop_block

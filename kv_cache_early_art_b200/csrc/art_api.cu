@@ -27,6 +27,9 @@ using art_host::is_null;
 struct Problem {
     int dtype;
     int B, Hq, Hkv, G, d, page, max_blocks, num_pages;
+    // query tokens sharing one walk; G = NQ * GQ rows per unit
+    int NQ = 1, GQ = 0;
+    int64_t q_st = 0, out_st = 0, stop_st = 0;
 };
 
 art_status_t check_tensors(const art_params_t *p, Problem *pr)
@@ -93,6 +96,53 @@ art_status_t check_tensors(const art_params_t *p, Problem *pr)
     pr->num_pages = (int)NP;
     if ((int64_t)B * Hkv > (int64_t)INT32_MAX / 16)
         return ART_ERR_SHAPE;
+    return ART_OK;
+}
+
+// Several query tokens per sequence: q and out are [B, T, Hq, d], stop_block
+// [B, T, Hkv].  Token 0's slices go through the single-query checks; the
+// token dimension is checked here.
+art_status_t check_tensors_multi(const art_params_t *p, int nq, Problem *pr)
+{
+    const art_tensor_t *q = &p->q, *o = &p->out, *st = &p->stop_block;
+    if (is_null(q) || is_null(o) || is_null(st))
+        return ART_ERR_NULL;
+    if (q->ndim != 4 || o->ndim != 4 || st->ndim != 3)
+        return ART_ERR_SHAPE;
+    if (q->shape[1] != nq || o->shape[1] != nq || st->shape[1] != nq)
+        return ART_ERR_SHAPE;
+    art_params_t v = *p;
+    auto drop_token_dim = [](const art_tensor_t &t, art_tensor_t *r) {
+        *r = t;
+        r->ndim = t.ndim - 1;
+        r->shape[0] = t.shape[0];
+        r->stride[0] = t.stride[0];
+        for (int i = 1; i < r->ndim; ++i) {
+            r->shape[i] = t.shape[i + 1];
+            r->stride[i] = t.stride[i + 1];
+        }
+        for (int i = r->ndim; i < 4; ++i) {
+            r->shape[i] = 0;
+            r->stride[i] = 0;
+        }
+    };
+    drop_token_dim(*q, &v.q);
+    drop_token_dim(*o, &v.out);
+    drop_token_dim(*st, &v.stop_block);
+    art_status_t s = check_tensors(&v, pr);
+    if (s != ART_OK)
+        return s;
+    const int64_t es = elem_size(q->dtype);
+    if (q->stride[1] < 0 || (q->stride[1] * es) % 16 || o->stride[1] < 0 || st->stride[1] < 0)
+        return ART_ERR_SHAPE;
+    if (nq > 1 && ((int64_t)nq * pr->G > 8 || pr->d != 128))
+        return ART_ERR_UNSUPPORTED;  // every token's heads must fit one unit's eight rows
+    pr->NQ = nq;
+    pr->GQ = pr->G;
+    pr->G = nq * pr->G;
+    pr->q_st = q->stride[1];
+    pr->out_st = o->stride[1];
+    pr->stop_st = st->stride[1];
     return ART_OK;
 }
 
@@ -181,6 +231,29 @@ KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax, int nmw)
     if (gmax == 1) return pick_dp<__nv_bfloat16, art::kEngineCuda, 1, 1>(d, page);
     if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineCuda, 4, 1>(d, page);
     return pick_dp<__nv_bfloat16, art::kEngineCuda, 8, 1>(d, page);
+}
+
+// Two query tokens per walk (head dim 128): bf16 on the tensor-core engine,
+// fp32 on the CUDA-core engine.
+template <typename T, int ENGINE, int GMAX, int NMW>
+KernelFn pick_page_multi(int page)
+{
+    return page == 16 ? art::art_walk_kernel<T, 128, 16, GMAX, ENGINE, NMW, 2>
+                      : art::art_walk_kernel<T, 128, 64, GMAX, ENGINE, NMW, 2>;
+}
+
+KernelFn pick_kernel_multi(int dtype, int engine, int page, int gmax, int nmw)
+{
+    if (dtype == ART_F32)
+        return gmax == 4 ? pick_page_multi<float, art::kEngineCuda, 4, 1>(page)
+                         : pick_page_multi<float, art::kEngineCuda, 8, 1>(page);
+    if (engine != art::kEngineMma)
+        return nullptr;
+    if (nmw == 4)
+        return gmax == 4 ? pick_page_multi<__nv_bfloat16, art::kEngineMma, 4, 4>(page)
+                         : pick_page_multi<__nv_bfloat16, art::kEngineMma, 8, 4>(page);
+    return gmax == 4 ? pick_page_multi<__nv_bfloat16, art::kEngineMma, 4, 1>(page)
+                     : pick_page_multi<__nv_bfloat16, art::kEngineMma, 8, 1>(page);
 }
 
 // ------------------------------------------------------ device caches ----
@@ -396,10 +469,11 @@ art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const Device
     return ART_OK;
 }
 
-art_status_t launch(const art_params_t *p, art_stream_t stream)
+// tokens_dim: q and out are [B, T, Hq, d] and stop_block [B, T, Hkv] (T = nq)
+art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool tokens_dim = false)
 {
     Problem pr;
-    art_status_t st = check_tensors(p, &pr);
+    art_status_t st = tokens_dim ? check_tensors_multi(p, nq, &pr) : check_tensors(p, &pr);
     if (st != ART_OK)
         return st;
     st = check_params(p);
@@ -414,21 +488,26 @@ art_status_t launch(const art_params_t *p, art_stream_t stream)
     Shape s;
     if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
         return st;
-    KernelFn fn = pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw);
+    KernelFn fn = nq == 1 ? pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw)
+                          : pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw);
+    if (!fn)
+        return ART_ERR_UNSUPPORTED;
     if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
         return st;
 
     KernelArgs ka;
     std::memset(&ka, 0, sizeof ka);
+    // with several tokens the head stride is the one after the token dimension
+    const int hd = tokens_dim ? 2 : 1;
     ka.q = p->q.data;
     ka.q_sb = p->q.stride[0];
-    ka.q_sh = p->q.stride[1];
+    ka.q_sh = p->q.stride[hd];
     ka.out = static_cast<float *>(p->out.data);
     ka.out_sb = p->out.stride[0];
-    ka.out_sh = p->out.stride[1];
+    ka.out_sh = p->out.stride[hd];
     ka.stop_block = static_cast<int32_t *>(p->stop_block.data);
     ka.stop_sb = p->stop_block.stride[0];
-    ka.stop_sh = p->stop_block.stride[1];
+    ka.stop_sh = p->stop_block.stride[hd];
     ka.page_table = static_cast<const int32_t *>(p->page_table.data);
     ka.pt_sb = p->page_table.stride[0];
     ka.block_order = static_cast<const int32_t *>(p->block_order.data);
@@ -454,6 +533,11 @@ art_status_t launch(const art_params_t *p, art_stream_t stream)
     ka.max_blocks = pr.max_blocks;
     ka.timeout_ns = p->timeout_ns > 0 ? p->timeout_ns : 2000000000LL;
     ka.debug_flags = p->debug_flags;
+    ka.NQ = pr.NQ;
+    ka.GQ = nq == 1 ? pr.G : pr.GQ;
+    ka.q_st = pr.q_st;
+    ka.out_st = pr.out_st;
+    ka.stop_st = pr.stop_st;
 
     if ((st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
         return st;
@@ -510,6 +594,15 @@ art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
     if (!p)
         return ART_ERR_NULL;
     return launch(p, stream);
+}
+
+art_status_t art_decode_attention_multi(const art_params_t *p, int32_t n_queries, art_stream_t stream)
+{
+    if (!p)
+        return ART_ERR_NULL;
+    if (n_queries != 1 && n_queries != 2)
+        return ART_ERR_UNSUPPORTED;
+    return launch(p, stream, n_queries, true);
 }
 
 art_status_t art_decode_attention(const art_tensor_t *q, const art_tensor_t *k_cache, const art_tensor_t *v_cache,

@@ -42,6 +42,7 @@ constexpr uint32_t kEndOfStream = 0xFFFFFFFFu;
 constexpr int kMaxThreads = 352;  // producer + up to 4 merge + up to 6 compute warps
 constexpr int kMaxComputeWarps = 6;
 constexpr int kMinWindow = 8;     // at least one merge batch
+constexpr int kRedFloats = 2 * 4 * 40;  // merge-warp exchange buffer
 constexpr int kErrTimeout = -7;
 constexpr int kErrBadIndex = -8;
 constexpr int kEngineCuda = 1;
@@ -71,6 +72,10 @@ struct KernelArgs {
     int32_t PF;                         // pages pulled into L2 ahead of the staged loads
     int64_t timeout_ns;
     int32_t debug_flags;
+    // several query tokens per sequence sharing one walk (NQ = 1: one query);
+    // G = NQ * GQ rows per unit, row r is head r % GQ of token r / GQ
+    int32_t NQ, GQ;
+    int64_t q_st, out_st, stop_st;      // element strides between a sequence's tokens
 };
 
 // Shared-memory carve-up, identical on host and device.
@@ -98,7 +103,7 @@ __host__ __device__ inline Layout make_layout(int S, int NW, int R, int page, in
     L.pbuf_off = off;
     off += pbuf ? (uint32_t)(NW * page * gmax * 4) : 0u;
     L.red_off = off;
-    off += 2 * 4 * 34 * 4 + 16;  // merge-warp exchange: 2 batches x up to 4 warps x (32 sums, flag, norm),
+    off += kRedFloats * 4 + 16;  // merge-warp exchange: 2 batches x up to 4 warps x (32 sums, flag, norms),
                                  // then the batch size merge warp 0 chose, per batch parity
     L.meta_off = off;
     off += 2 * S * 4;  // stage_j[S], stage_nv[S]
@@ -483,6 +488,19 @@ struct CudaEngine {
             for (int e = 0; e < DE; ++e)
                 qf[g][e] = (g < a.G) ? to_f32<T>(qp[(int64_t)(h * a.G + g) * a.q_sh + lane * DE + e]) : 0.f;
     }
+    // several tokens per unit: row g is head g % GQ of token g / GQ
+    __device__ void load_q_rows(const KernelArgs &a, int b, int h, int lane)
+    {
+        const T *qp = reinterpret_cast<const T *>(a.q) + (int64_t)b * a.q_sb;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+            const int t = g / a.GQ, gg = g - t * a.GQ;
+            const T *row = qp + (int64_t)t * a.q_st + (int64_t)(h * a.GQ + gg) * a.q_sh;
+#pragma unroll
+            for (int e = 0; e < DE; ++e)
+                qf[g][e] = (g < a.G) ? to_f32<T>(row[lane * DE + e]) : 0.f;
+        }
+    }
 
     // returns false on abort
     __device__ bool block(const KernelArgs &a, const Shared &sh, int s, uint32_t par, int nv, float *pbuf,
@@ -618,6 +636,24 @@ struct MmaEngine {
             qb[ks][1] = 0u;
             if (r < a.G) {
                 const __nv_bfloat16 *row = qp + (int64_t)(h * a.G + r) * a.q_sh + ks * 16 + 2 * c;
+                qb[ks][0] = *reinterpret_cast<const uint32_t *>(row);
+                qb[ks][1] = *reinterpret_cast<const uint32_t *>(row + 8);
+            }
+        }
+    }
+    // several tokens per unit: row r is head r % GQ of token r / GQ
+    __device__ void load_q_rows(const KernelArgs &a, int b, int h, int lane)
+    {
+        const int r = lane >> 2, c = lane & 3;
+        const int t = r / a.GQ, g = r - t * a.GQ;
+        const __nv_bfloat16 *qp = reinterpret_cast<const __nv_bfloat16 *>(a.q) + (int64_t)b * a.q_sb +
+                                  (int64_t)t * a.q_st + (int64_t)(h * a.GQ + g) * a.q_sh;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qb[ks][0] = 0u;
+            qb[ks][1] = 0u;
+            if (r < a.G) {
+                const __nv_bfloat16 *row = qp + ks * 16 + 2 * c;
                 qb[ks][0] = *reinterpret_cast<const uint32_t *>(row);
                 qb[ks][1] = *reinterpret_cast<const uint32_t *>(row + 8);
             }
@@ -1274,9 +1310,452 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = failed ? -1 : stop;
 }
 
+// Several query tokens of one sequence sharing one walk: NQ tokens of GQ
+// heads each, G = NQ * GQ rows in the block states.  The blocks are folded
+// as in merge_role; what differs is that every token keeps its own
+// statistics (over its own GQ * d outputs), patience counter and stop.  The
+// sums of o.Delta, |Delta|^2 and |o|^2 are split by token, the patience rule
+// runs once per token, and a token that has stopped is frozen: its rows get
+// beta = 0 for every later block, so its output stays the prefix output at
+// its own stop (a stop inside a batch replays the batch with the stopped
+// token's later blocks weighted 0).  Each token's stop and output are those
+// of its own single-query walk; the walk ends when every token has stopped.
+// KB = 16 / NQ blocks per batch, so that the (block, token) sums fill the
+// 32 lanes of one reduce-scatter.
+template <int D, int GMAX, int ENGINE, int NMW, int NQ>
+__device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, int h, int N, int mw)
+{
+    using MS = MergeShape<D, GMAX, ENGINE, NMW>;
+    using Lay = typename MS::Lay;
+    constexpr int NVW = MS::NVW, VW = Lay::VW, VP = VW / 2, NM = MS::NM;
+    constexpr int KB = 16 / NQ;                  // blocks per batch
+    constexpr int KH = 32 / GMAX;                // blocks per row of scan lanes
+    constexpr int NH = KB > KH ? KB / KH : 1;    // (block, row) entries per scan lane
+    constexpr int RS = 32 + 1 + NQ;              // exchange floats per merge warp: sums, flag, norms
+    constexpr uint32_t ALL = (1u << NQ) - 1u;
+    static_assert(NQ == 2 || NQ == 4, "tokens per walk");
+    static_assert(NH * KH >= KB && NH <= 2, "scan rows");
+    static_assert(2 * 4 * RS <= kRedFloats, "exchange buffer");
+    const int lane = threadIdx.x & 31;
+    const int G = a.G, GQ = a.GQ;
+    const float eps_m = a.eps_m_arr ? a.eps_m_arr[b] : a.eps_m;
+    const float eps_d = a.eps_d_arr ? a.eps_d_arr[b] : a.eps_d;
+    const int P = a.P_arr ? a.P_arr[b] : a.P;
+    const int minb = a.minb_arr ? a.minb_arr[b] : a.min_blocks;
+    const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
+    const uint32_t u_off = sh.L.u_off_floats;
+    const int slot_floats = (int)(sh.L.slot_bytes / 4);
+    const int vbase = mw * NVW;
+
+    // scan lane: blocks kl (and kl + KH) of the batch, row gl of token tok_gl
+    const int kl = lane / GMAX, gl = lane % GMAX;
+    const int tok_gl = gl < G ? gl / GQ : NQ;
+    // token of the low and high half of each packed pair this lane keeps
+    // (NQ for padding rows, which never count)
+    int tlo[NVW], thi[NVW];
+#pragma unroll
+    for (int ii = 0; ii < NVW; ++ii) {
+        const int r0 = Lay::head(lane, vbase + ii, 0), r1 = Lay::head(lane, vbase + ii, 1);
+        tlo[ii] = r0 < G ? r0 / GQ : NQ;
+        thi[ii] = r1 < G ? r1 / GQ : NQ;
+    }
+    float Mx = -CUDART_INF_F, Lm = 0.f;
+    uint64_t o[NVW][VP];
+#pragma unroll
+    for (int i = 0; i < NVW; ++i)
+#pragma unroll
+        for (int q = 0; q < VP; ++q)
+            o[i][q] = 0ull;
+
+    int cnt[NQ], stop[NQ];
+#pragma unroll
+    for (int t = 0; t < NQ; ++t) {
+        cnt[t] = 0;
+        stop[t] = 0;
+    }
+    uint32_t done = 0u;  // bit t: token t has stopped (the same in every lane)
+    bool failed = false;
+    if (a.debug_flags & 1) {
+        if (!warp_wait<true>(sh.never(a.S, a.R), 0u, sh.abort, a.timeout_ns, a.device_status))
+            failed = true;
+    }
+
+    auto load_u = [&](const float *sp, uint64_t (&uv)[NVW][VP]) {
+#pragma unroll
+        for (int ii = 0; ii < NVW; ++ii) {
+            const float *up = sp + u_off + Lay::off(lane, vbase + ii);
+            if constexpr (VW == 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(up);
+                uv[ii][0] = pk2(x.x, x.y);
+                uv[ii][1] = pk2(x.z, x.w);
+            } else {
+                const float2 x = *reinterpret_cast<const float2 *>(up);
+                uv[ii][0] = pk2(x.x, x.y);
+            }
+        }
+    };
+    // split packed per-vector sums by token: entry t of out gets the halves of token t
+    auto by_token = [&](const uint64_t (&x)[NVW], float (&out)[NQ]) {
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+            float acc = 0.f;
+#pragma unroll
+            for (int ii = 0; ii < NVW; ++ii) {
+                acc += tlo[ii] == t ? lo2(x[ii]) : 0.f;
+                acc += thi[ii] == t ? hi2(x[ii]) : 0.f;
+            }
+            out[t] = acc;
+        }
+    };
+    // fold batch block k into this warp's slice; with sums, v[2 (k NQ + t)]
+    // and v[2 (k NQ + t) + 1] get token t's o.Delta and |Delta|^2 of the slice
+    auto fold = [&](int k, float beta, const uint64_t (&uv)[NVW][VP], float (&v)[32], bool sums) {
+        uint64_t bp[NVW];
+        const int kr = NH > 1 ? k % KH : k;
+        if constexpr (Lay::kTwoHeads) {
+            const int h0 = Lay::head(lane, 0, 0);
+            const float b0 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0);
+            const float b1 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0 + 1);
+#pragma unroll
+            for (int ii = 0; ii < NVW; ++ii)
+                bp[ii] = pk2(b0, b1);
+        } else {
+#pragma unroll
+            for (int ii = 0; ii < NVW; ++ii) {
+                const float bi = __shfl_sync(0xffffffffu, beta, kr * GMAX + vbase + ii);
+                bp[ii] = (vbase + ii < G) ? pk2(bi, bi) : 0ull;
+            }
+        }
+        uint64_t sd[NVW], se[NVW];
+#pragma unroll
+        for (int ii = 0; ii < NVW; ++ii) {
+            sd[ii] = 0ull;
+            se[ii] = 0ull;
+#pragma unroll
+            for (int q = 0; q < VP; ++q) {
+                const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
+                if (sums) {
+                    sd[ii] = fma2(o[ii][q], dl, sd[ii]);
+                    se[ii] = fma2(dl, dl, se[ii]);
+                }
+                o[ii][q] = add2(o[ii][q], dl);
+            }
+        }
+        if (sums) {
+            float pd[NQ], pe[NQ];
+            by_token(sd, pd);
+            by_token(se, pe);
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) {
+                v[2 * (k * NQ + t)] = pd[t];
+                v[2 * (k * NQ + t) + 1] = pe[t];
+            }
+        }
+    };
+    auto fold_batch = [&](int s0, int kend, float beta, float beta_hi, float (&v)[32], bool sums) {
+        uint64_t ua[NVW][VP], ub[NVW][VP];
+        load_u(sh.ring + (size_t)s0 * slot_floats, ua);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            if (k > kend)
+                break;
+            if (k + 1 <= kend) {
+                int sn = s0 + k + 1;
+                sn = sn >= a.R ? sn - a.R : sn;
+                load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
+            }
+            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, (k & 1) ? ub : ua, v, sums);
+        }
+    };
+
+    int s0 = 0;
+    uint32_t ph0 = 0;
+    for (int j0 = 0, batch = 0; !failed && done != ALL && j0 < N; ++batch) {
+        const int nmax = min(KB, N - j0);
+        // 1. wait for the batch (as in merge_role)
+        int sk = s0 + (lane < KB ? lane : 0);
+        uint32_t pk = ph0;
+        if (sk >= a.R) {
+            sk -= a.R;
+            pk ^= 1u;
+        }
+        const float *spk = sh.ring + (size_t)sk * slot_floats;
+        bool local_fail = false;
+        int nb = 0;
+        if (mw == 0) {
+            uint64_t t0 = 0;
+            for (uint32_t it = 0;; ++it) {
+                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk, a.S), pk);
+                if (__any_sync(0xffffffffu, arrived && __float_as_uint(spk[0]) != 0u)) {
+                    local_fail = true;
+                    break;
+                }
+                if (__all_sync(0xffffffffu, arrived || lane >= nmax)) {
+                    nb = nmax;
+                    break;
+                }
+                if ((it & 7u) == 7u) {
+                    int quit = 0;
+                    if (lane == 0) {
+                        const uint64_t now = global_timer_ns();
+                        if (t0 == 0)
+                            t0 = now;
+                        if (*sh.abort) {
+                            quit = 1;
+                        } else if ((int64_t)(now - t0) > a.timeout_ns) {
+                            *sh.abort = 1u;
+                            record_error(a.device_status, kErrTimeout);
+                            quit = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, quit, 0)) {
+                        local_fail = true;
+                        break;
+                    }
+                }
+            }
+        }
+        if constexpr (NM > 1) {
+            volatile int *agreed = reinterpret_cast<volatile int *>(sh.red + kRedFloats) + (batch & 1);
+            if (mw == 0 && lane == 0)
+                *agreed = local_fail ? -1 : nb;
+            merge_barrier2(NM * 32);
+            const int vv = *agreed;
+            local_fail = vv < 0;
+            nb = vv < 0 ? 0 : vv;
+        }
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            v[q] = 0.f;
+        float beta = 0.f, beta_hi = 0.f;
+        float n0part[NQ];
+#pragma unroll
+        for (int t = 0; t < NQ; ++t)
+            n0part[t] = 0.f;
+        uint64_t o0[NVW][VP];
+        if (!local_fail) {
+            // 2. shares of the softmax mass per row; rows of stopped tokens get 0
+            float mk[NH], lk[NH];
+            float Mb = Mx;
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+                const int k = kl + hh * KH;
+                mk[hh] = -CUDART_INF_F;
+                lk[hh] = 0.f;
+                if (k < nb && gl < G) {
+                    int sl = s0 + k;
+                    sl = sl >= a.R ? sl - a.R : sl;
+                    const float *sp = sh.ring + (size_t)sl * slot_floats;
+                    mk[hh] = sp[4 + gl];
+                    lk[hh] = sp[4 + GMAX + gl];
+                }
+                Mb = fmaxf(Mb, mk[hh]);
+            }
+#pragma unroll
+            for (int off = GMAX; off < 32; off <<= 1)
+                Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
+            float w[NH], S[NH];
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+                w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : lk[hh] * ex2_approx(mk[hh] - Mb);
+                S[hh] = w[hh];
+            }
+#pragma unroll
+            for (int off = GMAX; off < 32; off <<= 1)
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh) {
+                    const float t = __shfl_up_sync(0xffffffffu, S[hh], off);
+                    if (lane >= off)
+                        S[hh] += t;
+                }
+            if constexpr (NH > 1)
+                S[1] += __shfl_sync(0xffffffffu, S[0], (KH - 1) * GMAX + gl);
+            const float base = (Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb);
+            const bool frozen = tok_gl < NQ && ((done >> tok_gl) & 1u);
+            float Lam[NH], bh[NH];
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+                Lam[hh] = base + S[hh];
+                bh[hh] = (Lam[hh] > 0.f && !frozen) ? w[hh] * rcp_approx(Lam[hh]) : 0.f;
+            }
+            beta = bh[0];
+            beta_hi = bh[NH - 1];
+            const float Llast = (NH > 1 && nb - 1 >= KH) ? Lam[NH - 1] : Lam[0];
+            Lm = __shfl_sync(0xffffffffu, Llast, ((nb - 1) % KH) * GMAX + gl);
+            Mx = Mb;
+            // 3. per-token ||o||^2 before the batch, then fold the batch
+            uint64_t n2[NVW];
+#pragma unroll
+            for (int i = 0; i < NVW; ++i) {
+                n2[i] = 0ull;
+#pragma unroll
+                for (int q = 0; q < VP; ++q) {
+                    o0[i][q] = o[i][q];
+                    n2[i] = fma2(o[i][q], o[i][q], n2[i]);
+                }
+            }
+            by_token(n2, n0part);
+            fold_batch(s0, nb - 1, beta, beta_hi, v, true);
+        }
+        // 4. lane l: warp sum of entry l = 2 (k NQ + t) + q
+        reduce_scatter32(v, lane);
+#pragma unroll
+        for (int t = 0; t < NQ; ++t)
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                n0part[t] += __shfl_xor_sync(0xffffffffu, n0part[t], off);
+        float *red = sh.red + (batch & 1) * (NM * RS);
+        red[mw * RS + lane] = v[0];
+        if (lane == 0) {
+            reinterpret_cast<volatile int *>(red)[mw * RS + 32] = local_fail ? 1 : 0;
+#pragma unroll
+            for (int t = 0; t < NQ; ++t)
+                red[mw * RS + 33 + t] = n0part[t];
+        }
+        if constexpr (NM > 1)
+            merge_barrier(NM * 32);
+        else
+            __syncwarp();
+        bool any_fail = false;
+        float tot = 0.f, n0b[NQ];
+#pragma unroll
+        for (int t = 0; t < NQ; ++t)
+            n0b[t] = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NM; ++w2) {
+            any_fail |= reinterpret_cast<volatile int *>(red)[w2 * RS + 32] != 0;
+            tot += red[w2 * RS + lane];
+#pragma unroll
+            for (int t = 0; t < NQ; ++t)
+                n0b[t] += red[w2 * RS + 33 + t];
+        }
+        if (any_fail) {
+            failed = true;
+            break;
+        }
+        // 5. statistics of (block k, token t) in lane 2 (k NQ + t); the prefix
+        //    over k of token t runs over lanes 2 NQ apart
+        const int tl = (lane >> 1) % NQ;
+        const float Dp = tot;
+        const float Ep = __shfl_down_sync(0xffffffffu, tot, 1);
+        const float tt = 2.f * Dp + Ep;
+        float pre = tt;
+#pragma unroll
+        for (int off = 2 * NQ; off < 32; off <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, pre, off);
+            if (lane >= off)
+                pre += u;
+        }
+        float n0base = n0b[0];
+#pragma unroll
+        for (int t = 1; t < NQ; ++t)
+            n0base = tl == t ? n0b[t] : n0base;
+        const float n0 = n0base + (pre - tt);
+        const float n1sq = n0 + tt;
+        bool stable = false;
+        if (n0 > 0.f && n1sq > 0.f) {
+            const float i0 = rsqrtf(n0), i1 = rsqrtf(n1sq);
+            const float r0 = n0 * i0, r1 = n1sq * i1;
+            const float d_scale = __fdividef(fabsf(tt), (r1 + r0) * r0);
+            const float pr = Dp * i0;
+            const float x = r0 + pr;
+            const float y2 = fmaxf(Ep - pr * pr, 0.f);
+            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : 1.f - x * i1;
+            stable = (d_scale < eps_m) && (d_dir < eps_d);
+        }
+        // 6. patience per token, one lane per block (as in merge_role)
+        const int kq = lane & (KB - 1);
+        int kstop[NQ];
+        bool replay = false;
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+            const bool stab_k = __shfl_sync(0xffffffffu, stable, 2 * (kq * NQ + t)) && (j0 + kq >= 1);
+            const uint32_t sbits = __ballot_sync(0xffffffffu, lane < nb && stab_k);
+            const uint32_t zeros = ~sbits & ((2u << kq) - 1u);
+            const int run = zeros == 0u ? cnt[t] + kq + 1 : kq - (31 - __clz(zeros));
+            const uint32_t hit = __ballot_sync(0xffffffffu, lane < nb && run >= P && j0 + kq + 1 >= minb);
+            const int run_last = __shfl_sync(0xffffffffu, run, nb - 1);
+            kstop[t] = -1;
+            if (!((done >> t) & 1u)) {
+                cnt[t] = run_last;
+                if (hit) {
+                    kstop[t] = __ffs(hit) - 1;
+                    stop[t] = j0 + kstop[t] + 1;
+                    replay |= kstop[t] < nb - 1;
+                }
+            }
+        }
+        if (replay) {
+            // fold the batch again from the snapshot, each token that stopped
+            // inside it weighted 0 after its stop block
+#pragma unroll
+            for (int i = 0; i < NVW; ++i)
+#pragma unroll
+                for (int q = 0; q < VP; ++q)
+                    o[i][q] = o0[i][q];
+            int ks = NQ > 0 ? kstop[0] : -1;
+#pragma unroll
+            for (int t = 1; t < NQ; ++t)
+                ks = tok_gl == t ? kstop[t] : ks;
+            if (tok_gl < NQ && ks >= 0) {
+                if (kl > ks)
+                    beta = 0.f;
+                if (kl + KH > ks)
+                    beta_hi = 0.f;
+            }
+            fold_batch(s0, nb - 1, beta, beta_hi, v, false);
+        }
+        int maxstop = 0;
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+            if (kstop[t] >= 0)
+                done |= 1u << t;
+            maxstop = max(maxstop, stop[t]);
+        }
+        if (mw == 0 && lane == 0)
+            st_relaxed_cluster_u32(ctrl_cl, done == ALL ? (kStopBit | (uint32_t)maxstop) : (uint32_t)(j0 + nb));
+        j0 += nb;
+        s0 += nb;
+        if (s0 >= a.R) {
+            s0 -= a.R;
+            ph0 ^= 1u;
+        }
+    }
+    if (!failed) {
+#pragma unroll
+        for (int t = 0; t < NQ; ++t)
+            if (!((done >> t) & 1u))
+                stop[t] = N;
+    }
+    if (failed && mw == 0 && lane == 0)
+        st_relaxed_cluster_u32(ctrl_cl, kStopBit);
+    float *op = a.out + (int64_t)b * a.out_sb;
+#pragma unroll
+    for (int ii = 0; ii < NVW; ++ii)
+#pragma unroll
+        for (int e = 0; e < VW; ++e) {
+            const int i = vbase + ii;
+            const int r = Lay::head(lane, i, e);
+            const float val = (e & 1) ? hi2(o[ii][e >> 1]) : lo2(o[ii][e >> 1]);
+            if (r < G && (Lay::kTwoHeads || i < G)) {
+                const int t = r / GQ, g = r - t * GQ;
+                op[(int64_t)t * a.out_st + (int64_t)(h * GQ + g) * a.out_sh + Lay::dim(lane, i, e)] =
+                    failed ? 0.f : val;
+            }
+        }
+    if (mw == 0) {
+#pragma unroll
+        for (int t = 0; t < NQ; ++t)
+            if (lane == t)
+                a.stop_block[(int64_t)b * a.stop_sb + (int64_t)t * a.stop_st + (int64_t)h * a.stop_sh] =
+                    failed ? -1 : stop[t];
+    }
+}
+
 // ---- kernel ------------------------------------------------------------------------
 
-template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW>
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW, int NQ = 1>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv)
@@ -1318,8 +1797,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             first_lb = a.block_order ? __ldg(a.block_order + (int64_t)b * a.bo_sb + jj) : (jj == 0 ? 0 : N - jj);
     }
     EngineFor<T, D, PAGE, GMAX, ENGINE> eng;
-    if (walk && warp > NM)
-        eng.load_q(a, b, h, threadIdx.x & 31);
+    if (walk && warp > NM) {
+        if constexpr (NQ == 1)
+            eng.load_q(a, b, h, threadIdx.x & 31);
+        else
+            eng.load_q_rows(a, b, h, threadIdx.x & 31);
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.S; ++s) {
@@ -1344,20 +1827,31 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         if (warp == 0)
             producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank, first_lb, first_pp);
         else if (warp <= NM) {
-            if (rank == 0)
-                merge_role<D, GMAX, ENGINE, NMW>(a, sh, b, h, N, warp - 1);
+            if (rank == 0) {
+                if constexpr (NQ == 1)
+                    merge_role<D, GMAX, ENGINE, NMW>(a, sh, b, h, N, warp - 1);
+                else
+                    merge_role_multi<D, GMAX, ENGINE, NMW, NQ>(a, sh, b, h, N, warp - 1);
+            }
         } else
             compute_role<T, D, PAGE, GMAX, ENGINE>(a, sh, b, h, warp - 1 - NM, eng);
     } else if (rank == 0 && warp == 1) {
         const int lane = threadIdx.x & 31;
         float *op = a.out + (int64_t)b * a.out_sb;
-        for (int i = lane; i < a.G * D; i += 32)
-            op[(int64_t)(h * a.G + i / D) * a.out_sh + i % D] = 0.f;
-        if (lane == 0) {
-            a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = bad_len ? -1 : 0;
-            if (bad_len)
-                record_error(a.device_status, kErrBadIndex);
+        if constexpr (NQ == 1) {
+            for (int i = lane; i < a.G * D; i += 32)
+                op[(int64_t)(h * a.G + i / D) * a.out_sh + i % D] = 0.f;
+        } else {
+            for (int i = lane; i < a.G * D; i += 32) {
+                const int r = i / D, t = r / a.GQ, g = r - t * a.GQ;
+                op[(int64_t)t * a.out_st + (int64_t)(h * a.GQ + g) * a.out_sh + i % D] = 0.f;
+            }
         }
+        if (lane < NQ)
+            a.stop_block[(int64_t)b * a.stop_sb + (int64_t)lane * a.stop_st + (int64_t)h * a.stop_sh] =
+                bad_len ? -1 : 0;
+        if (lane == 0 && bad_len)
+            record_error(a.device_status, kErrBadIndex);
     }
     __syncwarp();
     cluster_sync();  // remote stores into the leader are complete

@@ -53,7 +53,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["Workload", "CONFIGS", "make_workload", "make_custom", "sink_recency_order", "streaming_subset"]
+__all__ = ["Workload", "CONFIGS", "make_workload", "make_custom", "sink_recency_order", "streaming_subset",
+           "draft_queries", "token_view"]
 
 
 @dataclass
@@ -346,3 +347,25 @@ def streaming_subset(w: Workload, window_blocks: int, sink_blocks: int = 1, name
     return Workload(name or f"{w.name}_stream{window_blocks}", w.q, w.k_cache, w.v_cache, new_pt.to(dev),
                     order.to(dev), new_len.to(torch.int32).to(dev), w.eps_m, w.eps_d, w.P, w.min_blocks,
                     w.page, dict(w.meta, pruned=f"sinks {sink_blocks} + window {window_blocks} pages"))
+
+
+def draft_queries(w: Workload, T: int, spread: float = 0.5, seed: int = 0) -> torch.Tensor:
+    """Queries of T decode tokens per sequence, [B, T, Hq, d] in the cache's
+    dtype: token 0 is w.q, token t > 0 is w.q + spread * N(0, 1) drawn in
+    fp32 from a CPU generator seeded with seed * 131 + t (neighbouring draft
+    tokens of one sequence ask similar questions), then rounded to the
+    cache dtype."""
+    q0 = w.q.detach().cpu().to(torch.float32)
+    toks = [q0]
+    for t in range(1, int(T)):
+        g = torch.Generator().manual_seed(int(seed) * 131 + t)
+        toks.append(q0 + float(spread) * torch.randn(q0.shape, generator=g, dtype=torch.float32))
+    q = torch.stack(toks, dim=1).to(w.k_cache.dtype)
+    return q.to(w.q.device)
+
+
+def token_view(w: Workload, q_multi: torch.Tensor, t: int) -> Workload:
+    """The single-query workload of token t: w with q = q_multi[:, t]."""
+    v = w.to(w.q.device)
+    v.q = q_multi[:, t].contiguous().to(w.q.device)
+    return v

@@ -225,3 +225,43 @@ def test_importance_binding_refuses_cpu_tensors(art):
     with pytest.raises(ValueError):
         art.art_build_order_importance(torch.zeros(2, 8, 128), torch.zeros(10, 2, 128), z,
                                        torch.zeros(2, dtype=torch.int32), 64)
+
+
+def multi_params(art, B=2, T_=2, Hq=8, Hkv=2, d=128, page=64, NP=10, MB=5, dt=1):
+    """art_params_t for art_decode_attention_multi over fake (never read) buffers."""
+    import kv_cache_early_art_b200 as pkg
+    p = pkg.ArtParams()
+    p.q = T([B, T_, Hq, d], dt)
+    p.k_cache, p.v_cache = T([NP, Hkv, page, d], dt), T([NP, Hkv, page, d], dt)
+    p.page_table, p.seq_lens = T([B, MB], 2), T([B], 2)
+    p.out, p.stop_block = T([B, T_, Hq, d], 0), T([B, T_, Hkv], 2)
+    p.eps_m, p.eps_d, p.P, p.min_blocks = 1e-3, 1e-4, 2, 1
+    return p
+
+
+def test_multi_query_host_errors(art):
+    lib = art.raw_library()
+    lib.art_decode_attention_multi.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    r = lambda p, n=2: lib.art_decode_attention_multi(ctypes.addressof(p), n, None)
+    assert lib.art_decode_attention_multi(None, 2, None) == -1
+    assert r(multi_params(art), 3) == -4                      # only 1 or 2 tokens per walk
+    assert r(multi_params(art), 0) == -4
+    assert r(multi_params(art, T_=1), 2) == -2                # token dimension differs from n_queries
+    assert r(multi_params(art, Hq=10, Hkv=2)) == -4           # 2 tokens x 5 heads > 8 rows
+    assert r(multi_params(art, d=64)) == -4                   # head dim 128 only
+    p = multi_params(art)
+    p.q.ndim = 3
+    assert r(p) == -2                                         # q must be [B, T, Hq, d]
+    p = multi_params(art)
+    p.out.shape[1] = 3
+    assert r(p) == -2                                         # token count differs
+    p = multi_params(art)
+    p.stop_block.shape[2] = 3
+    assert r(p) == -2                                         # stop_block [B, T, Hkv]
+    p = multi_params(art)
+    p.q.stride[1] = 8 * 128 + 4                               # token stride not 16-byte aligned
+    p.q.stride[0] = 2 * p.q.stride[1]
+    assert r(p) == -2
+    p = multi_params(art)
+    p.k_cache.dtype = 0
+    assert r(p) == -3                                         # cache dtype differs from q
