@@ -447,7 +447,7 @@ def run_table(args):
     import torch
 
     import kv_cache_early_art_b200 as art
-    from kv_cache_early_art_b200.workloads import CONFIGS, make_workload, streaming_subset
+    from kv_cache_early_art_b200.workloads import CONFIGS, draft_queries, make_workload, streaming_subset
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -503,6 +503,43 @@ def run_table(args):
         print(json.dumps(row), flush=True)
         return row
 
+    pairs = []
+
+    def measure_pair(w):
+        """Two decode tokens per sequence (the second the first plus noise):
+        two separate single-query walks against one shared walk."""
+        qm = draft_queries(w, 2, seed=0)
+        kw = dict(eps_m_per_seq=w.eps_m, eps_d_per_seq=w.eps_d, P_per_seq=w.P, min_blocks_per_seq=w.min_blocks)
+        sep = [(torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev),
+                torch.empty(w.B, w.Hkv, dtype=torch.int32, device=dev),
+                torch.zeros(w.B * w.Hkv, dtype=torch.int32, device=dev)) for _ in range(2)]
+        q_tok = [qm[:, t].contiguous() for t in range(2)]
+
+        def separate():
+            for t in range(2):
+                art.art_decode_attention_ex(q_tok[t], w.k_cache, w.v_cache, w.page_table, w.block_order,
+                                            w.seq_lens, out=sep[t][0], stop_block=sep[t][1],
+                                            blocks_fetched=sep[t][2], **kw)
+        out2 = torch.empty(w.B, 2, w.Hq, w.d, dtype=torch.float32, device=dev)
+        stop2 = torch.empty(w.B, 2, w.Hkv, dtype=torch.int32, device=dev)
+        fetched2 = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device=dev)
+
+        def shared():
+            art.art_decode_attention_multi(qm, w.k_cache, w.v_cache, w.page_table, w.block_order, w.seq_lens,
+                                           out=out2, stop_block=stop2, blocks_fetched=fetched2, **kw)
+        separate()
+        shared()
+        ms_sep, ms_sh = median_ms(separate), median_ms(shared)
+        bb = 2 * w.page * w.d * w.k_cache.element_size()
+        f_sep = sum(int(x[2].sum().item()) for x in sep)
+        f_sh = int(fetched2.sum().item())
+        same = sum(int((stop2[:, t] != sep[t][1]).sum().item()) for t in range(2))
+        row = {"workload": w.name, "ms_separate": ms_sep, "ms_shared": ms_sh, "queries": 2 * w.B,
+               "consumed": int(stop2.clamp(min=0).sum().item()), "fetched_separate": f_sep, "fetched_shared": f_sh,
+               "gbs_shared": f_sh * bb / (ms_sh / 1e3) / 1e9, "stop_differs": same}
+        pairs.append(row)
+        print(json.dumps(row), flush=True)
+
     names = list(CONFIGS) if args.table == "all" else args.table.split(",")
     for name in names:
         base = make_workload(name, device=dev)
@@ -529,6 +566,8 @@ def run_table(args):
             row = measure(w, "ART, importance order", w.eps_m, w.eps_d, w.P, importance=bufs)
             row.update(summary_ms=sum_ms, order_ms=order_ms)
             print(json.dumps({"workload": w.name, "summary_ms": sum_ms, "order_ms": order_ms}), flush=True)
+            if w.d == 128 and 2 * w.G <= 8:      # two tokens fit one unit's eight rows
+                measure_pair(w)
         del base, variants
         torch.cuda.empty_cache()
     print("| workload | variant | walk ms | queries/s | blocks consumed / total | skipped | pages fetched | GB/s | of HBM |")
@@ -543,6 +582,15 @@ def run_table(args):
     for r in rows:
         if "summary_ms" in r:
             print(f"| {r['workload']} | {r['summary_ms']:.4f} | {r['order_ms']:.4f} |")
+    if pairs:
+        print()
+        print("| workload | two walks ms | one shared walk ms | speed-up | queries/s shared | pages fetched "
+              "(two walks / shared) | shared GB/s | stops differing |")
+        print("|---|---|---|---|---|---|---|---|")
+        for r in pairs:
+            print(f"| {r['workload']} | {r['ms_separate']:.4f} | {r['ms_shared']:.4f} | "
+                  f"{r['ms_separate'] / r['ms_shared']:.2f}x | {r['queries'] / (r['ms_shared'] / 1e3):.0f} | "
+                  f"{r['fetched_separate']} / {r['fetched_shared']} | {r['gbs_shared']:.0f} | {r['stop_differs']} |")
     return 0
 
 

@@ -259,7 +259,7 @@ KernelFn pick_kernel_multi(int dtype, int engine, int page, int gmax, int nmw)
 // ------------------------------------------------------ device caches ----
 
 struct DeviceInfo {
-    int sms = 0, smem_optin = 0;
+    int sms = 0, smem_optin = 0, smem_sm = 0, smem_reserved = 0;
 };
 
 std::mutex g_mu;
@@ -276,7 +276,9 @@ art_status_t device_info(DeviceInfo *out)
     if (it == g_dev.end()) {
         DeviceInfo di;
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
             return ART_ERR_LAUNCH;
         it = g_dev.emplace(dev, di).first;
     }
@@ -370,6 +372,9 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
     // with fewer units each unit is split over a cluster and needs a deeper
     // window to cover the latency from fetch to merged stop decision.
     static const int many_units[][3] = {{2, 2, 16}, {1, 2, 16}, {2, 2, 8}, {1, 2, 8}};
+    // many units whose state ring is too large for two CTAs per SM (eight
+    // rows per unit): one CTA per SM with the same pages in flight
+    static const int many_units_wide[][3] = {{4, 4, 16}, {3, 3, 16}, {2, 2, 16}, {1, 2, 8}};
     static const int few_units_large[][3] = {{5, 5, 28}, {4, 4, 24}, {2, 4, 24}, {3, 3, 24}, {2, 2, 24},
                                              {2, 4, 16}, {2, 2, 16}, {1, 2, 16}, {1, 2, 8}};
     static const int few_units_small[][3] = {{4, 8, 32}, {4, 8, 16}, {4, 4, 16}, {2, 4, 16}, {2, 2, 8},
@@ -379,6 +384,11 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
     if (units >= di.sms) {
         cand = many_units;
         ncand = 4;
+        Shape t = s;
+        t.NW = t.S = 2;
+        t.R = 16;
+        if (2 * (smem_bytes(t, pr) + di.smem_reserved) > di.smem_sm)
+            cand = many_units_wide;
     } else if (tile >= 16384) {
         cand = few_units_large;
         ncand = 9;
