@@ -498,8 +498,8 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     Shape s;
     if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
         return st;
-    KernelFn fn = nq == 1 ? pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw)
-                          : pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw);
+    KernelFn fn = nq > 1 ? pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw)
+                         : pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw);
     if (!fn)
         return ART_ERR_UNSUPPORTED;
     if ((st = prepare_kernel(fn, s.smem)) != ART_OK)

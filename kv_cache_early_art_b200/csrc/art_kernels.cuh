@@ -1012,7 +1012,12 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         }
         uint64_t sd = 0ull, se = 0ull;
 #pragma unroll
-        for (int ii = 0; ii < NVW; ++ii)
+        for (int ii = 0; ii < NVW; ++ii) {
+            // the CUDA-core engine writes no state for padding rows (vector
+            // i >= G): their slot floats are whatever the shared memory held,
+            // so they are skipped, not weighted by 0 (0 * inf is NaN)
+            if (!Lay::kTwoHeads && vbase + ii >= G)
+                continue;
 #pragma unroll
             for (int q = 0; q < VP; ++q) {
                 const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
@@ -1022,6 +1027,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 }
                 o[ii][q] = add2(o[ii][q], dl);
             }
+        }
         if (sums) {
             pd = lo2(sd) + hi2(sd);
             pe = lo2(se) + hi2(se);
@@ -1333,8 +1339,8 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
     constexpr int NH = KB > KH ? KB / KH : 1;    // (block, row) entries per scan lane
     constexpr int RS = 32 + 1 + NQ;              // exchange floats per merge warp: sums, flag, norms
     constexpr uint32_t ALL = (1u << NQ) - 1u;
-    static_assert(NQ == 2 || NQ == 4, "tokens per walk");
-    static_assert(NH * KH >= KB && NH <= 2, "scan rows");
+    static_assert(NQ == 1 || NQ == 2 || NQ == 4, "tokens per walk");
+    static_assert(NH * KH >= KB && NH <= 4, "scan rows");
     static_assert(2 * 4 * RS <= kRedFloats, "exchange buffer");
     const int lane = threadIdx.x & 31;
     const int G = a.G, GQ = a.GQ;
@@ -1431,6 +1437,8 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
         for (int ii = 0; ii < NVW; ++ii) {
             sd[ii] = 0ull;
             se[ii] = 0ull;
+            if (!Lay::kTwoHeads && vbase + ii >= G)
+                continue;  // padding rows: never written (see merge_role)
 #pragma unroll
             for (int q = 0; q < VP; ++q) {
                 const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
@@ -1452,7 +1460,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
             }
         }
     };
-    auto fold_batch = [&](int s0, int kend, float beta, float beta_hi, float (&v)[32], bool sums) {
+    auto fold_batch = [&](int s0, int kend, const float (&bh)[NH], float (&v)[32], bool sums) {
         uint64_t ua[NVW][VP], ub[NVW][VP];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
 #pragma unroll
@@ -1464,7 +1472,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, (k & 1) ? ub : ua, v, sums);
+            fold(k, bh[k / KH], (k & 1) ? ub : ua, v, sums);
         }
     };
 
@@ -1528,7 +1536,10 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
 #pragma unroll
         for (int q = 0; q < 32; ++q)
             v[q] = 0.f;
-        float beta = 0.f, beta_hi = 0.f;
+        float bh[NH];  // beta of scan entry hh: block kl + hh KH, row gl
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh)
+            bh[hh] = 0.f;
         float n0part[NQ];
 #pragma unroll
         for (int t = 0; t < NQ; ++t)
@@ -1569,19 +1580,27 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                     if (lane >= off)
                         S[hh] += t;
                 }
-            if constexpr (NH > 1)
-                S[1] += __shfl_sync(0xffffffffu, S[0], (KH - 1) * GMAX + gl);
+            // each row of scan lanes continues from the total of the rows before it
+            float carry = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+                S[hh] += carry;
+                if (hh + 1 < NH)
+                    carry = __shfl_sync(0xffffffffu, S[hh], (KH - 1) * GMAX + gl);
+            }
             const float base = (Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb);
             const bool frozen = tok_gl < NQ && ((done >> tok_gl) & 1u);
-            float Lam[NH], bh[NH];
+            float Lam[NH];
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) {
                 Lam[hh] = base + S[hh];
                 bh[hh] = (Lam[hh] > 0.f && !frozen) ? w[hh] * rcp_approx(Lam[hh]) : 0.f;
             }
-            beta = bh[0];
-            beta_hi = bh[NH - 1];
-            const float Llast = (NH > 1 && nb - 1 >= KH) ? Lam[NH - 1] : Lam[0];
+            const int hl = (nb - 1) / KH;  // row of the batch's last block
+            float Llast = Lam[0];
+#pragma unroll
+            for (int hh = 1; hh < NH; ++hh)
+                Llast = hl == hh ? Lam[hh] : Llast;
             Lm = __shfl_sync(0xffffffffu, Llast, ((nb - 1) % KH) * GMAX + gl);
             Mx = Mb;
             // 3. per-token ||o||^2 before the batch, then fold the batch
@@ -1596,7 +1615,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                 }
             }
             by_token(n2, n0part);
-            fold_batch(s0, nb - 1, beta, beta_hi, v, true);
+            fold_batch(s0, nb - 1, bh, v, true);
         }
         // 4. lane l: warp sum of entry l = 2 (k NQ + t) + q
         reduce_scatter32(v, lane);
@@ -1699,12 +1718,12 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
             for (int t = 1; t < NQ; ++t)
                 ks = tok_gl == t ? kstop[t] : ks;
             if (tok_gl < NQ && ks >= 0) {
-                if (kl > ks)
-                    beta = 0.f;
-                if (kl + KH > ks)
-                    beta_hi = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < NH; ++hh)
+                    if (kl + hh * KH > ks)
+                        bh[hh] = 0.f;
             }
-            fold_batch(s0, nb - 1, beta, beta_hi, v, false);
+            fold_batch(s0, nb - 1, bh, v, false);
         }
         int maxstop = 0;
 #pragma unroll
@@ -1755,6 +1774,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
 
 // ---- kernel ------------------------------------------------------------------------
 
+// NQ: query tokens sharing the walk (1: merge_role, else merge_role_multi).
 template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW, int NQ = 1>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,

@@ -279,3 +279,24 @@ def test_launch_shapes(cuda_lib, dtype, engine):
         assert torch.equal(out, out0), (cl, nw, st, win)
         assert_fetch_bound(w, stop, fetched, win + info["prefetch"])
     assert ran >= len(SHAPES[dtype]) - 1
+
+
+@pytest.mark.parametrize("dtype,G,d,page", [("bf16", 3, 128, 16), ("f32", 7, 64, 64), ("f32", 3, 128, 16),
+                                            ("bf16", 7, 128, 64)])
+def test_stale_shared_memory_is_ignored(cuda_lib, dtype, G, d, page):
+    """Every SM's shared memory is filled with NaN (then -inf) right before
+    the walk: a block state's padding rows (G below the engine's row count)
+    are never written, and the result must not depend on what they hold."""
+    from tests import smem_poison
+    rng = np.random.default_rng(500 + G)
+    lens = [int(x) for x in rng.integers(1, 40 * page, size=3)] + [page * 3, 1]
+    w = make_custom(B=len(lens), Hq=G * 2, Hkv=2, d=d, page=page, dtype=dtype, seq_lens=lens, seed=500 + G,
+                    keys="recency", planted=3, planted_gain=5.0, order="random", eps_m=2e-2, eps_d=2e-3,
+                    P=[1, 2, 3, 2, 1], min_blocks=[1, 3, 0, 2, 1])
+    for engine in ([1] if dtype == "f32" else [1, 2]):
+        for pattern in (smem_poison.NAN, smem_poison.NEG_INF):
+            smem_poison.poison(pattern)
+            out, stop, fetched, status, info = run_gpu(cuda_lib, w, engine=engine)
+            assert status == 0
+            parity.check(w, out, stop)
+            assert torch.isfinite(out).all()
