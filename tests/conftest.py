@@ -30,3 +30,16 @@ def cuda_lib():
     build.build_library()
     import kv_cache_early_art_b200 as art
     return art
+
+
+@pytest.fixture(autouse=True)
+def _poison_shared_memory(request):
+    """With ART_POISON_SMEM=nan or =neginf, every GPU test starts with all
+    shared memory filled with that pattern, so a kernel that reads shared
+    memory it never wrote gives a wrong (non-finite) result instead of
+    passing on whatever an earlier kernel left there."""
+    mode = os.environ.get("ART_POISON_SMEM", "")
+    if mode and request.node.get_closest_marker("gpu") is not None and gpu_available():
+        from tests import smem_poison
+        smem_poison.poison({"nan": smem_poison.NAN, "neginf": smem_poison.NEG_INF}[mode])
+    yield

@@ -150,3 +150,22 @@ def test_unsupported_combinations(cuda_lib):
     w5 = make_custom(B=1, Hq=10, Hkv=2, d=128, page=64, dtype="bf16", seq_lens=[300], seed=1)
     with pytest.raises(cuda_lib.ArtError, match="UNSUPPORTED"):
         run_multi(cuda_lib, w5, draft_queries(w5, 2, seed=1))   # 2 x 5 heads > 8 rows
+
+
+def test_shared_walk_ignores_stale_shared_memory(cuda_lib):
+    """Shared memory filled with NaN, then -inf, before each shared walk:
+    padding rows (3 heads per token, 6 of the engine's 8 rows used) are never
+    written and must not matter."""
+    from tests import smem_poison
+    w = make_custom(B=3, Hq=6, Hkv=2, d=128, page=16, dtype="bf16", seq_lens=[700, 333, 1000], seed=61, planted=2,
+                    planted_gain=5.0, eps_m=1e-2, eps_d=1e-3, P=2, min_blocks=1)
+    qm = draft_queries(w, 2, seed=61)
+    wf = make_custom(B=3, Hq=6, Hkv=2, d=128, page=16, dtype="f32", seq_lens=[700, 333, 1000], seed=62, planted=2,
+                     planted_gain=5.0, eps_m=1e-2, eps_d=1e-3, P=2, min_blocks=1)
+    qf = draft_queries(wf, 2, seed=62)
+    for ww, qq in ((w, qm), (wf, qf)):
+        for pattern in (smem_poison.NAN, smem_poison.NEG_INF):
+            smem_poison.poison(pattern)
+            out, stop, fetched, status, info = run_multi(cuda_lib, ww, qq)
+            assert status == 0 and torch.isfinite(out).all()
+            check_tokens(ww, qq, out, stop, fetched, info["window"] + info["prefetch"])
