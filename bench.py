@@ -285,16 +285,31 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     fetched = torch.zeros(B * Hkv, dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    out = torch.empty(B, w.Hq, d, dtype=torch.float32, device=dev)
-    stop = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    T = args.multi                                # decode tokens per sequence sharing one walk
+    if T > 1:
+        from kv_cache_early_art_b200.workloads import draft_queries
+        q_all = draft_queries(w, T, seed=0).to(dev)
+        out = torch.empty(B, T, w.Hq, d, dtype=torch.float32, device=dev)
+        stop = torch.empty(B, T, Hkv, dtype=torch.int32, device=dev)
+        entry = art.art_decode_attention_multi
+    else:
+        q_all = w.q
+        out = torch.empty(B, w.Hq, d, dtype=torch.float32, device=dev)
+        stop = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+        entry = art.art_decode_attention_ex
+
+    def walked(st):
+        """Blocks the walk consumed: per unit, the latest token's stop."""
+        st = st.clamp(min=0)
+        return int((st.amax(dim=1) if T > 1 else st).sum().item())
     flush = L2Flush(torch, dev)
 
     def step(eps_off=False):
         kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                   P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                   device_status=status, out=out, stop_block=stop)
-        return art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
-                                           eps_m=0.0, eps_d=0.0, want_info=True, **kw)
+        return entry(q_all, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
+                     eps_m=0.0, eps_d=0.0, want_info=True, **kw)
 
     def timed(n, eps_off=False):
         """n steps; per step: flush, then the walk between events.
@@ -306,8 +321,7 @@ def run_ours(args):
             kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                       P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                       device_status=status, out=out, stop_block=stop)
-            art.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
-                                        eps_m=0.0, eps_d=0.0, **kw)
+            entry(q_all, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens, eps_m=0.0, eps_d=0.0, **kw)
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -329,13 +343,13 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
     stops = stop.clone()
-    consumed = int(stops.clamp(min=0).sum().item())
+    consumed = walked(stops)
     fetched_blocks = int(fetched.sum().item())
     assert int(status.item()) == 0
     ms = sum(step_ms) / len(step_ms)
     ms_walk = sum(walk_ms) / len(walk_ms)
     ms_max = reduce_max(ms, ws, dev)
-    queries_all = reduce_sum(float(B), ws, dev)
+    queries_all = reduce_sum(float(B * T), ws, dev)
     value = queries_all / (ms_max / 1000.0)
 
     # ---- termination disabled: the same kernel as full attention ----
@@ -343,21 +357,26 @@ def run_ours(args):
         step(eps_off=True)
     f_step, f_walk = timed(max(3, args.steps // 4), eps_off=True)
     ms_full = sum(f_walk) / len(f_walk)
-    full_consumed = int(stop.clamp(min=0).sum().item())
+    full_consumed = walked(stop)
 
     alg_bytes = consumed * block_bytes
     fetch_bytes = fetched_blocks * block_bytes
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (ms_walk / 1000.0) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "traffic": ncu_traffic(args.workload), "peak_kind": peak_kind,
-            "kernel": "art_walk_kernel (the whole step: the order is built inside it)",
+            "traffic": ncu_traffic(args.workload if T == 1 else f"{args.workload}_shared{T}"),
+            "peak_kind": peak_kind,
+            "kernel": "art_walk_kernel (the whole step: the order is built inside it)" if T == 1 else
+                      f"art_walk_kernel, {T} tokens per walk (the whole step)",
             "algorithmic_bytes_per_launch": alg_bytes}
 
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": str(w.k_cache.dtype).replace("torch.", "").replace("bfloat16", "bf16"),
-            "data": "synthetic", "config": config_for(args.workload, w, ws),
+            "data": "synthetic", "config": dict(config_for(args.workload, w, ws), **(
+                {"queries_per_sequence": T, "queries": "draft tokens sharing one walk: token 0 the workload's "
+                 "query, token 1 that query plus 0.5 N(0,1); each token keeps its own ART decision"}
+                if T > 1 else {})),
             "kv_gbs_fetched": fetch_bytes / (ms_walk / 1000.0) / 1e9,
             "kv_gbs_algorithmic": achieved,
             "hbm_frac_of_measured": fetch_bytes / (ms_walk / 1000.0) / 1e9 / peak,
@@ -366,7 +385,7 @@ def run_ours(args):
             "fetch_waste_blocks": fetched_blocks - consumed,
             "walk_ms": ms_walk,
             "full_attention": {"walk_ms": ms_full, "kv_gbs": full_consumed * block_bytes / (ms_full / 1000.0) / 1e9,
-                               "queries_per_s": B / (ms_full / 1000.0),
+                               "queries_per_s": B * T / (ms_full / 1000.0),
                                "art_speedup": ms_full / ms_walk},
             "launch": info, "gpu_launches": args.steps,
             "roofline": roof, "clocks": clk.summary()}
@@ -385,7 +404,7 @@ def run_ours(args):
             blk = torch.empty(n, dtype=torch.uint8, device=device, pin_memory=pin)
             views = [blk[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for o, t in zip(offs, parts)]
             return blk, views
-        ins = [w.q, w.page_table, w.seq_lens]
+        ins = [q_all, w.page_table, w.seq_lens]
         in_h, (q_h, pt_h, sl_h) = carve(ins, pin=True)
         for hv, t in zip((q_h, pt_h, sl_h), ins):
             hv.copy_(t.cpu())
@@ -397,9 +416,8 @@ def run_ours(args):
 
         def e2e_step():
             in_d.copy_(in_h, non_blocking=True)
-            art.art_decode_attention_ex(q_d, w.k_cache, w.v_cache, pt_d, None, sl_d, eps_m_per_seq=w.eps_m,
-                                        eps_d_per_seq=w.eps_d, P_per_seq=w.P, min_blocks_per_seq=w.min_blocks,
-                                        out=out_v, stop_block=stop_v)
+            entry(q_d, w.k_cache, w.v_cache, pt_d, None, sl_d, eps_m_per_seq=w.eps_m, eps_d_per_seq=w.eps_d,
+                  P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, out=out_v, stop_block=stop_v)
             out_h.copy_(out_d, non_blocking=True)
 
         for _ in range(3):
@@ -603,6 +621,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--multi", type=int, default=1, choices=[1, 2],
+                    help="decode tokens per sequence sharing one walk (2: art_decode_attention_multi)")
     ap.add_argument("--cpu-seconds", type=float, default=5.0)
     ap.add_argument("--table", default=None, help="'all' or comma-separated workloads: per-workload table")
     ap.add_argument("--table-reps", type=int, default=20)
