@@ -993,16 +993,14 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     };
     // Fold batch block k into this warp's slice: Delta = beta (u - o),
     // o += Delta; with sums, add o.Delta and |Delta|^2 of the slice to pd, pe.
-    auto fold = [&](int k, float beta, const uint64_t (&uv)[NVW][VP], float &pd, float &pe, bool sums) {
+    auto fold = [&](int k, float beta, uint64_t bq, const uint64_t (&uv)[NVW][VP], float &pd, float &pe,
+                    bool sums) {
         uint64_t bp[NVW];
         const int kr = NH > 1 ? k % KH : k;  // row of the scan lanes holding block k
-        if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads
-            const int h0 = Lay::head(lane, 0, 0);
-            const float b0 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0);
-            const float b1 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0 + 1);
+        if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads: bq = (beta, beta) of both
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii)
-                bp[ii] = pk2(b0, b1);
+                bp[ii] = bq;
         } else {  // vector i holds head i
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii) {
@@ -1037,6 +1035,20 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     auto fold_batch = [&](int s0, int kend, float beta, float beta_hi, float (&v)[16], bool sums) {
         uint64_t ua[NVW][VP], ub[NVW][VP];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
+        // the beta pairs of every block of the batch, fetched before the fold
+        // so that the shuffles stay off the chain that carries o from block to block
+        uint64_t bq[KB];
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            bq[k] = 0ull;
+            if constexpr (Lay::kTwoHeads) {
+                const float bk = (NH > 1 && k >= KH) ? beta_hi : beta;
+                const int kr = NH > 1 ? k % KH : k;
+                const int h0 = Lay::head(lane, 0, 0);
+                bq[k] = pk2(__shfl_sync(0xffffffffu, bk, kr * GMAX + h0),
+                            __shfl_sync(0xffffffffu, bk, kr * GMAX + h0 + 1));
+            }
+        }
 #pragma unroll
         for (int k = 0; k < KB; ++k) {
             if (k > kend)
@@ -1046,7 +1058,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
+            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, bq[k], (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
         }
     };
 
