@@ -1427,16 +1427,13 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
     };
     // fold batch block k into this warp's slice; with sums, v[2 (k NQ + t)]
     // and v[2 (k NQ + t) + 1] get token t's o.Delta and |Delta|^2 of the slice
-    auto fold = [&](int k, float beta, const uint64_t (&uv)[NVW][VP], float (&v)[32], bool sums) {
+    auto fold = [&](int k, float beta, uint64_t bq, const uint64_t (&uv)[NVW][VP], float (&v)[32], bool sums) {
         uint64_t bp[NVW];
         const int kr = NH > 1 ? k % KH : k;
-        if constexpr (Lay::kTwoHeads) {
-            const int h0 = Lay::head(lane, 0, 0);
-            const float b0 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0);
-            const float b1 = __shfl_sync(0xffffffffu, beta, kr * GMAX + h0 + 1);
+        if constexpr (Lay::kTwoHeads) {  // bq: the block's beta pair, fetched before the fold
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii)
-                bp[ii] = pk2(b0, b1);
+                bp[ii] = bq;
         } else {
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii) {
@@ -1475,6 +1472,17 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
     auto fold_batch = [&](int s0, int kend, const float (&bh)[NH], float (&v)[32], bool sums) {
         uint64_t ua[NVW][VP], ub[NVW][VP];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
+        uint64_t bq[KB];  // as in merge_role: every block's beta pair before the fold
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            bq[k] = 0ull;
+            if constexpr (Lay::kTwoHeads) {
+                const int kr = NH > 1 ? k % KH : k;
+                const int h0 = Lay::head(lane, 0, 0);
+                bq[k] = pk2(__shfl_sync(0xffffffffu, bh[k / KH], kr * GMAX + h0),
+                            __shfl_sync(0xffffffffu, bh[k / KH], kr * GMAX + h0 + 1));
+            }
+        }
 #pragma unroll
         for (int k = 0; k < KB; ++k) {
             if (k > kend)
@@ -1484,7 +1492,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            fold(k, bh[k / KH], (k & 1) ? ub : ua, v, sums);
+            fold(k, bh[k / KH], bq[k], (k & 1) ? ub : ua, v, sums);
         }
     };
 
