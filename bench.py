@@ -71,11 +71,18 @@ def measured_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the walk's sources with comments and blank lines removed, so
+    that a comment edit does not void an ncu record taken on the same code."""
+    import re
     h = hashlib.sha256()
     for rel in ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
                 "kv_cache_early_art_b200/csrc/art_api.cu"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        src = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+        h.update(src.encode())
     return h.hexdigest()[:16]
 
 

@@ -901,7 +901,8 @@ struct MergeLayout<D, GMAX, kEngineMma> {  // tensor-core slots: vector v = dt*W
 
 // How the merge is split: NM warps share the output elements (vectors
 // [mw*NVW, mw*NVW+NVW) of every lane belong to merge warp mw); KB blocks are
-// folded per batch, with one scan lane per (block, head) pair.
+// folded per batch; a scan lane holds one (block, head) pair, or two when
+// eight heads fill a row of 32 lanes at four blocks.
 template <int D, int GMAX, int ENGINE, int NMW>
 struct MergeShape {
     using Lay = MergeLayout<D, GMAX, ENGINE>;
@@ -930,9 +931,10 @@ __device__ __forceinline__ void merge_barrier2(int nthreads)
 }
 
 // Folds block states into the running output in walk order, KB blocks per
-// batch.  Per batch: wait for the KB states; one lane per (block, head) forms
-// the blocks' shares of the softmax mass with a prefix scan (block max, then
-// prefix sums of l 2^(m - M)); every merge warp folds the blocks into its
+// batch.  Per batch: wait for the KB states; the scan lanes (one or two
+// (block, head) pairs each) form the blocks' shares of the softmax mass with
+// a prefix scan (block max, then prefix sums of l 2^(m - M)); every merge
+// warp folds the blocks into its
 // slice of o, accumulating ||o_{j-1}||^2, o_{j-1}.Delta_j and ||Delta_j||^2;
 // the slices' sums meet in shared memory; every merge warp then evaluates the
 // statistics of the batch's blocks lane-parallel and runs the patience rule,
