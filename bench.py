@@ -30,7 +30,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "ART decode-attn queries/s; KV GB/s read & % of B200 HBM peak; % KV blocks skipped"
-DEFAULT_WORKLOAD = "llama8b_b8"
+DEFAULT_WORKLOAD = "llama8b_b32"
 WORKLOAD_TEXT = {
     "tiny_fp32": "tiny fp32: B=1, Hq=Hkv=4, d=64, L=1024, 16-token blocks, 4 planted tokens",
     "llama8b_b8": "Llama-3-8B-shaped GQA 32/8, d=128, bf16 paged KV, B=8, L=8192, 64-token pages, "
@@ -71,16 +71,23 @@ def measured_peaks():
 
 
 def kernel_source_hash():
-    """Hash of the walk's sources with comments and blank lines removed, so
-    that a comment edit does not void an ncu record taken on the same code."""
+    """Hash of what the walk kernel is built from -- its sources, the host
+    header they include and the build script with its nvcc flags -- with
+    comments and blank lines removed, so that a comment edit does not void an
+    ncu record taken on the same code, while a change of code or flags does."""
     import re
     h = hashlib.sha256()
     for rel in ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
-                "kv_cache_early_art_b200/csrc/art_api.cu"):
+                "kv_cache_early_art_b200/csrc/art_api.cu", "kv_cache_early_art_b200/csrc/art_host.h",
+                "kv_cache_early_art_b200/build.py"):
         with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
             src = f.read()
-        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-        src = re.sub(r"//[^\n]*", "", src)
+        if rel.endswith(".py"):
+            src = re.sub(r'"""(?:.|\n)*?"""', "", src)
+            src = re.sub(r"#[^\n]*", "", src)
+        else:
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
         src = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
         h.update(src.encode())
     return h.hexdigest()[:16]
@@ -198,27 +205,44 @@ def reduce_sum(value: float, world: int, device=None) -> float:
 # ---------------------------------------------------------------- oracle ----
 
 def time_oracle(w_cpu, budget_s: float, ncores: int = 0):
-    """The CPU oracle on the whole batch, repeated until budget_s has passed
-    (ncores threads; 0: every host core)."""
+    """The CPU oracle on a bounded sample of the batch: groups of sequences
+    (enough kv-head units to give every thread one), cycling through the
+    batch, until budget_s has passed (ncores threads; 0: every host core).
+    Returns (queries/s, threads used, sequences timed, seconds)."""
     import oracle
     ncores = ncores or os.cpu_count() or 1
-    reps, t0 = 0, time.perf_counter()
+    per = max(1, -(-ncores // w_cpu.Hkv))           # sequences per call
+    groups = [sequences(w_cpu, list(range(b, min(b + per, w_cpu.B)))) for b in range(0, w_cpu.B, per)]
+    used = min(ncores, per * w_cpu.Hkv)
+    done, i, t0 = 0, 0, time.perf_counter()
     while True:
-        oracle.run(w_cpu, want_out=True, nthreads=ncores)
-        reps += 1
+        g = groups[i % len(groups)]
+        oracle.run(g, want_out=True, nthreads=ncores)
+        done += g.B
+        i += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return w_cpu.B * reps / el, ncores, reps, el
+    return done / el, used, done, el
+
+
+def sequences(w, seqs):
+    """The listed sequences of a CPU workload, sharing its caches."""
+    v = w.to("cpu")
+    sl = torch_index(seqs)
+    v.q, v.page_table, v.block_order, v.seq_lens = w.q[sl], w.page_table[sl], w.block_order[sl], w.seq_lens[sl]
+    v.eps_m, v.eps_d, v.P, v.min_blocks = w.eps_m[sl], w.eps_d[sl], w.P[sl], w.min_blocks[sl]
+    return v
+
+
+def torch_index(seqs):
+    import torch
+    return torch.as_tensor(seqs, dtype=torch.long)
 
 
 def one_sequence(w, b):
     """Sequence b of a CPU workload, sharing its caches (the oracle's sample)."""
-    v = w.to("cpu")
-    sl = slice(b, b + 1)
-    v.q, v.page_table, v.block_order, v.seq_lens = w.q[sl], w.page_table[sl], w.block_order[sl], w.seq_lens[sl]
-    v.eps_m, v.eps_d, v.P, v.min_blocks = w.eps_m[sl], w.eps_d[sl], w.P[sl], w.min_blocks[sl]
-    return v
+    return sequences(w, [b])
 
 
 def run_reference(args):
@@ -453,11 +477,12 @@ def run_ours(args):
     # ---- CPU oracle baseline (rank 0, N = 1) ----
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         w_cpu = w.to("cpu")
-        qps, cores, reps, el = time_oracle(w_cpu, args.cpu_seconds)
-        qps1, _, reps1, el1 = time_oracle(w_cpu, args.cpu_seconds / 2, ncores=1)
+        qps, cores, nseq, el = time_oracle(w_cpu, args.cpu_seconds)
+        qps1, _, nseq1, el1 = time_oracle(w_cpu, args.cpu_seconds / 2, ncores=1)
         line["cpu_baseline"] = {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                                "sample": f"whole {args.workload} batch ({w.B} queries) x {reps} in {el:.1f} s",
-                                "one_core": {"value": qps1, "sample": f"the same batch x {reps1} in {el1:.1f} s"}}
+                                "sample": f"{nseq} {args.workload} sequences (decode queries, every kv head), "
+                                          f"cycling through the batch, in {el:.1f} s",
+                                "one_core": {"value": qps1, "sample": f"{nseq1} sequences in {el1:.1f} s"}}
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -633,7 +658,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--multi", type=int, default=1, choices=[1, 2],
                     help="decode tokens per sequence sharing one walk (2: art_decode_attention_multi)")
-    ap.add_argument("--cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--table", default=None, help="'all' or comma-separated workloads: per-workload table")
     ap.add_argument("--table-reps", type=int, default=20)
     args = ap.parse_args(argv)

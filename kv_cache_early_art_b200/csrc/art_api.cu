@@ -396,13 +396,25 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         cand = few_units_small;
         ncand = 6;
     }
+    // every compute warp owns the same stages (stage i goes to warp i % NW),
+    // so S must be a multiple of NW: only a caller who fixes both can break that
+    if (p->compute_warps && p->stages && p->stages % p->compute_warps != 0)
+        return ART_ERR_PARAM;
     for (int i = 0; i < ncand; ++i) {
-        const int NW = p->compute_warps ? p->compute_warps : cand[i][0];
+        int NW = p->compute_warps ? p->compute_warps : cand[i][0];
         int S = p->stages ? p->stages : cand[i][1];
-        if (!p->stages && S < NW)
-            S = NW;
-        if (S % NW != 0 || S < NW)
-            return ART_ERR_PARAM;
+        if (p->stages && !p->compute_warps) {
+            // stages fixed, warps automatic: the largest warp count up to the
+            // candidate's that divides the stages
+            while (S % NW != 0)
+                --NW;
+        } else if (!p->stages) {
+            // warps fixed (or both automatic): round the candidate's stages up
+            // to a multiple of the warps, and down again past the 8-stage limit
+            S = NW * ((S + NW - 1) / NW);
+            if (S > 8)
+                S = NW * (8 / NW);
+        }
         s.NW = NW;
         s.S = S;
         s.R = p->window ? p->window : cand[i][2];

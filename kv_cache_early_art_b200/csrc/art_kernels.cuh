@@ -1823,7 +1823,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int unit = blockIdx.x / a.C;
     const int b = unit / a.Hkv, h = unit % a.Hkv;
     const int Lseq = a.seq_lens[b];
-    const int N = Lseq <= 0 ? 0 : (Lseq + PAGE - 1) / PAGE;
+    // (written so that lengths near INT32_MAX do not overflow: they are
+    // longer than any page table and reported below)
+    const int N = Lseq <= 0 ? 0 : Lseq / PAGE + (Lseq % PAGE != 0);
     const bool bad_len = N > a.max_blocks;
 
     constexpr int NM = MergeShape<D, GMAX, ENGINE, NMW>::NM;
@@ -1909,7 +1911,7 @@ __global__ void art_build_order_kernel(const int32_t *seq_lens, int B, int page,
     if (b >= B)
         return;
     const int L = seq_lens[b];
-    const int N = L <= 0 ? 0 : (L + page - 1) / page;
+    const int N = L <= 0 ? 0 : L / page + (L % page != 0);
     for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < max_blocks; j += gridDim.x * blockDim.x)
         order[(int64_t)b * row_stride + j] = j < N ? (j == 0 ? 0 : N - j) : -1;
 }

@@ -123,7 +123,9 @@ __device__ __forceinline__ void report(int32_t *status, int32_t code)
         atomicCAS(status, 0, code);
 }
 
-__device__ __forceinline__ int n_blocks_of(int L, int page) { return L <= 0 ? 0 : (L + page - 1) / page; }
+// blocks of a sequence of L tokens, without the overflow of (L + page - 1)
+// near INT32_MAX
+__device__ __forceinline__ int n_blocks_of(int L, int page) { return L <= 0 ? 0 : L / page + (L % page != 0); }
 
 // ------------------------------------------------------------ summary ----
 

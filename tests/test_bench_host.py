@@ -5,7 +5,8 @@ import shutil
 import bench
 
 SOURCES = ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
-           "kv_cache_early_art_b200/csrc/art_api.cu")
+           "kv_cache_early_art_b200/csrc/art_api.cu", "kv_cache_early_art_b200/csrc/art_host.h",
+           "kv_cache_early_art_b200/build.py")
 
 
 def _copy_sources(tmp_path):
@@ -26,3 +27,33 @@ def test_kernel_hash_ignores_comments_not_code(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == h0
     k.write_text(src.replace("kMinWindow = 8", "kMinWindow = 9", 1))
     assert bench.kernel_source_hash() != h0
+
+
+def test_kernel_hash_covers_build_flags_and_host_header(tmp_path, monkeypatch):
+    """A different nvcc flag or a change of the host header the walk is built
+    with voids the record; a docstring or comment edit in the build script
+    does not."""
+    _copy_sources(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    b = tmp_path / SOURCES[4]
+    src = b.read_text()
+    b.write_text('"""another docstring"""\n# a comment\n' + src)
+    assert bench.kernel_source_hash() == h0
+    b.write_text(src.replace('"-O3"', '"-O2"', 1))
+    assert bench.kernel_source_hash() != h0
+    b.write_text(src)
+    hh = tmp_path / SOURCES[3]
+    hh.write_text(hh.read_text() + "\ninline int extra_helper() { return 1; }\n")
+    assert bench.kernel_source_hash() != h0
+
+
+def test_oracle_sample_is_bounded():
+    """The CPU baseline times groups of sequences until its budget passes,
+    never a whole large batch at once."""
+    from kv_cache_early_art_b200.workloads import make_custom
+    w = make_custom(B=5, Hq=8, Hkv=2, d=32, page=8, dtype="f32", seq_lens=[40, 9, 64, 1, 30], seed=3)
+    qps, used, done, el = bench.time_oracle(w, 0.05, ncores=3)
+    assert used == 3 and done >= 2 and qps > 0
+    g = bench.sequences(w, [1, 3])
+    assert g.B == 2 and g.seq_lens.tolist() == [9, 1]

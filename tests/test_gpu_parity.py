@@ -216,28 +216,63 @@ def test_invalid_arguments_launch_nothing(cuda_lib):
 
 # ------------------------------------------------------------ full sizes ----
 
-def _full(art, name, seqs, engine=0):
+def _full(art, name, seqs=None, engine=0, **params):
+    """A named workload at its full size, in the launch configuration the
+    bench times (library-chosen shape, default order built inside the walk):
+    every unit (or the listed sequences) against the oracle.  params
+    overrides the per-sequence thresholds / patience (scalars)."""
     torch.manual_seed(0)
     w = make_workload(name, device="cuda")
-    out, stop, fetched, status, info = run_gpu(art, w, engine=engine)
-    assert status == 0
-    wc = parity.subset_sequences(w, seqs)
-    idx = torch.as_tensor(seqs)
-    s = parity.check(wc, out[idx], stop[idx])
+    for key, val in params.items():
+        dt = torch.int32 if key in ("P", "min_blocks") else torch.float32
+        setattr(w, key, torch.full((w.B,), val, dtype=dt, device="cuda"))
+    g = w
+    fetched = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, stop, info = art.art_decode_attention_ex(
+        g.q, g.k_cache, g.v_cache, g.page_table, None, g.seq_lens, eps_m_per_seq=g.eps_m, eps_d_per_seq=g.eps_d,
+        P_per_seq=g.P, min_blocks_per_seq=g.min_blocks, blocks_fetched=fetched, device_status=status,
+        engine=engine, want_info=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    fetched = fetched.view(w.B, w.Hkv)
+    if seqs is None:
+        wc, o, st = w.to("cpu"), out, stop
+    else:
+        wc = parity.subset_sequences(w, seqs)
+        idx = torch.as_tensor(seqs)
+        o, st = out[idx], stop[idx]
+    s = parity.check(wc, o, st)
     assert_fetch_bound(w, stop, fetched, info["window"] + info["prefetch"])
-    return s
+    return s, w, stop
 
 
 def test_llama8b_b32_full_size(cuda_lib):
-    _full(cuda_lib, "llama8b_b32", [0, 9, 20, 31])
+    """Every one of the 256 units of the B=32, L=32768 batch."""
+    _full(cuda_lib, "llama8b_b32")
+
+
+def test_llama8b_b32_eps0_full_size(cuda_lib):
+    """The full-attention companion of the same batch (eps_m = eps_d = 0):
+    every unit walks all 512 blocks and equals the oracle's full softmax."""
+    s, w, stop = _full(cuda_lib, "llama8b_b32", eps_m=0.0, eps_d=0.0)
+    N = w.n_blocks().cpu().numpy()[:, None]
+    assert (stop.cpu().numpy() == N).all()
+    assert s["blocks_consumed"] == s["blocks_total"]
 
 
 def test_qwen7b_b4_full_size(cuda_lib):
-    _full(cuda_lib, "qwen7b_b4", [0, 1, 2, 3])
+    _full(cuda_lib, "qwen7b_b4")
 
 
 def test_mistral7b_b128_full_size(cuda_lib):
-    _full(cuda_lib, "mistral7b_b128", list(range(0, 128, 9)))
+    """Every one of the 1024 units of the ragged B=128 batch, per-sequence
+    thresholds and patience."""
+    _full(cuda_lib, "mistral7b_b128")
+
+
+def test_llama8b_b8_full_size_default_order(cuda_lib):
+    _full(cuda_lib, "llama8b_b8")
 
 
 SHAPES = {
