@@ -79,7 +79,9 @@ def kernel_source_hash():
     h = hashlib.sha256()
     for rel in ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
                 "kv_cache_early_art_b200/csrc/art_api.cu", "kv_cache_early_art_b200/csrc/art_host.h",
-                "kv_cache_early_art_b200/build.py"):
+                "kv_cache_early_art_b200/csrc/art_walk.h", "kv_cache_early_art_b200/csrc/art_walk_f32.cu",
+                "kv_cache_early_art_b200/csrc/art_walk_bf16.cu", "kv_cache_early_art_b200/csrc/art_walk_mma.cu",
+                "kv_cache_early_art_b200/csrc/art_walk_multi.cu", "kv_cache_early_art_b200/build.py"):
         with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
             src = f.read()
         if rel.endswith(".py"):
@@ -336,14 +338,16 @@ def run_ours(args):
         return int((st.amax(dim=1) if T > 1 else st).sum().item())
     flush = L2Flush(torch, dev)
 
-    def step(eps_off=False):
+    def step(eps_off=False, det_off=False):
         kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                   P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                   device_status=status, out=out, stop_block=stop)
+        if det_off:
+            kw["detector_off"] = 1
         return entry(q_all, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
                      eps_m=0.0, eps_d=0.0, want_info=True, **kw)
 
-    def timed(n, eps_off=False):
+    def timed(n, eps_off=False, det_off=False):
         """n steps; per step: flush, then the walk between events.
         Returns per-step ms (twice: the whole step is the walk)."""
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
@@ -353,6 +357,8 @@ def run_ours(args):
             kw = dict(eps_m_per_seq=None if eps_off else w.eps_m, eps_d_per_seq=None if eps_off else w.eps_d,
                       P_per_seq=w.P, min_blocks_per_seq=w.min_blocks, blocks_fetched=fetched,
                       device_status=status, out=out, stop_block=stop)
+            if det_off:
+                kw["detector_off"] = 1
             entry(q_all, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens, eps_m=0.0, eps_d=0.0, **kw)
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
@@ -375,6 +381,7 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
     stops = stop.clone()
+    art_out = out.clone()
     consumed = walked(stops)
     fetched_blocks = int(fetched.sum().item())
     assert int(status.item()) == 0
@@ -390,6 +397,7 @@ def run_ours(args):
     f_step, f_walk = timed(max(3, args.steps // 4), eps_off=True)
     ms_full = sum(f_walk) / len(f_walk)
     full_consumed = walked(stop)
+    det = detector_overhead(args, T, step, timed, out, stop, torch, dev)
 
     alg_bytes = consumed * block_bytes
     fetch_bytes = fetched_blocks * block_bytes
@@ -419,6 +427,7 @@ def run_ours(args):
             "full_attention": {"walk_ms": ms_full, "kv_gbs": full_consumed * block_bytes / (ms_full / 1000.0) / 1e9,
                                "queries_per_s": B * T / (ms_full / 1000.0),
                                "art_speedup": ms_full / ms_walk},
+            "detector_overhead": det,
             "launch": info, "gpu_launches": args.steps,
             "roofline": roof, "clocks": clk.summary()}
 
@@ -466,7 +475,7 @@ def run_ours(args):
             b_.synchronize()
             e_ms.append(a.elapsed_time(b_))
         # the staged path computed what the device-resident one did
-        if not (torch.equal(out_hv, out.cpu()) and torch.equal(stop_hv, stop.cpu())):
+        if not (torch.equal(out_hv, art_out.cpu()) and torch.equal(stop_hv, stops.cpu())):
             raise RuntimeError("end-to-end result differs from the device-resident walk")
         em = reduce_max(sum(e_ms) / len(e_ms), ws, dev)
         line["e2e"] = {"value": queries_all / (em / 1000.0), "unit": "queries/s", "h2d_bytes_per_step": h2d,
@@ -489,6 +498,35 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def detector_overhead(args, T, step, timed, out, stop, torch, dev):
+    """The ART explainer's section 4 ablation (detector cost with termination
+    disabled): the walk at eps = 0, which forms every statistic and runs the
+    patience rule but never stops, against the same walk built without the
+    detector (detector_off), whose output must equal it bit for bit.  Rounds
+    of the two alternate; each round's median step time, best round kept."""
+    if T > 1:
+        return None
+    step(eps_off=True)
+    ref_out, ref_stop = out.clone(), stop.clone()
+    try:
+        step(det_off=True)
+    except Exception as e:           # not built for this shape
+        return {"unavailable": str(e)}
+    torch.cuda.synchronize(dev)
+    identical = bool(torch.equal(out, ref_out) and torch.equal(stop, ref_stop))
+    n = max(5, min(200, args.steps // 8))
+    med = lambda xs: sorted(xs)[len(xs) // 2]
+    eps0, off = [], []
+    for _ in range(4):
+        eps0.append(med(timed(n, eps_off=True)[1]))
+        off.append(med(timed(n, det_off=True)[1]))
+    a, b = min(eps0), min(off)
+    return {"eps0_walk_ms": a, "detector_off_walk_ms": b, "overhead_frac": a / b - 1.0,
+            "output_identical": identical, "rounds": 4, "steps_per_round": n,
+            "note": "eps = 0 walk (statistics and patience formed, never stopping) against the walk built "
+                    "without the detector; alternating rounds, median per round, best round"}
 
 
 def run_table(args):

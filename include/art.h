@@ -142,6 +142,18 @@ typedef struct {
     int32_t prefetch;              /* 0 or -1 off, else 1..64 blocks pulled into L2         */
                                    /* ahead of the staged loads.  Pages read past the stop  */
                                    /* stay below window + prefetch blocks.                  */
+    int32_t detector_off;          /* 0; 1 runs the walk without the ART detector: no      */
+                                   /* statistic, no patience rule, every block consumed     */
+                                   /* (stop_block = N_b).  The output equals the eps = 0    */
+                                   /* walk's bit for bit.  A timing reference for the cost  */
+                                   /* of the detector (the explainer's section 4 reports    */
+                                   /* it with termination disabled); thresholds, P and      */
+                                   /* min_blocks are ignored.  Built for BF16 caches on the */
+                                   /* tensor-core engine with d = 128 and 64-token pages,   */
+                                   /* and for F32 caches with d = 64, 16-token pages and    */
+                                   /* at most 4 query heads per kv head; other cases return */
+                                   /* ART_ERR_UNSUPPORTED, as does art_decode_attention_multi*/
+                                   /* with n_queries = 2.                                   */
 } art_params_t;
 
 /*

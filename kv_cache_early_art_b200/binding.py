@@ -56,7 +56,8 @@ class ArtParams(ctypes.Structure):
         ("blocks_fetched", ctypes.c_void_p), ("device_status", ctypes.c_void_p),
         ("engine", ctypes.c_int32), ("cluster_size", ctypes.c_int32), ("stages", ctypes.c_int32),
         ("compute_warps", ctypes.c_int32), ("window", ctypes.c_int32), ("timeout_ns", ctypes.c_int64),
-        ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo)), ("prefetch", ctypes.c_int32)]
+        ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo)), ("prefetch", ctypes.c_int32),
+        ("detector_off", ctypes.c_int32)]
 
 
 _P = ctypes.POINTER
@@ -146,7 +147,7 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
 
 def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P, min_blocks,
             sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status,
-            engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch):
+            engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch, detector_off=0):
     """Fill art_params_t (argument marshalling only); returns (params, info)."""
     per = [eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status]
     _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, *per)
@@ -170,6 +171,7 @@ def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_bl
     p.compute_warps, p.window, p.timeout_ns = int(compute_warps), int(window), int(timeout_ns)
     p.debug_flags = int(debug_flags)
     p.prefetch = int(prefetch)
+    p.detector_off = int(detector_off)
     info = ArtLaunchInfo()
     p.info = ctypes.pointer(info)
     return p, info
@@ -179,7 +181,8 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
                             P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                             P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                             engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                            debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None, want_info=False):
+                            debug_flags=0, prefetch=0, detector_off=0, out=None, stop_block=None, stream=None,
+                            want_info=False):
     """art_decode_attention_ex in art.h.  Per-sequence arrays are device
     tensors of length B (float32 thresholds, int32 P / min_blocks).
     Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
@@ -191,7 +194,7 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch)
+                      timeout_ns, debug_flags, prefetch, detector_off)
     st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
     _check(st, "art_decode_attention_ex")
     if want_info:
@@ -203,7 +206,7 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
                                P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                                P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                                engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                               debug_flags=0, prefetch=0, out=None, stop_block=None, stream=None,
+                               debug_flags=0, prefetch=0, detector_off=0, out=None, stop_block=None, stream=None,
                                want_info=False):
     """art_decode_attention_multi in art.h: q [B, T, Hq, d], T query tokens
     per sequence sharing one walk.  Returns (out [B, T, Hq, d],
@@ -216,7 +219,7 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch)
+                      timeout_ns, debug_flags, prefetch, detector_off)
     st = _lib.art_decode_attention_multi(ctypes.byref(p), int(T), _stream(stream))
     _check(st, "art_decode_attention_multi")
     if want_info:

@@ -12,10 +12,25 @@
 #include "../../include/art.h"
 #include "art_host.h"
 #include "art_kernels.cuh"
+#include "art_walk.h"
 
 namespace {
 
 using art::KernelArgs;
+
+// Default walk order: [0, N-1, N-2, ..., 1], -1 beyond N.
+__global__ void art_build_order_kernel(const int32_t *seq_lens, int B, int page, int32_t *order, int64_t row_stride,
+                                       int max_blocks)
+{
+    const int b = blockIdx.y;
+    if (b >= B)
+        return;
+    const int L = seq_lens[b];
+    const int N = L <= 0 ? 0 : L / page + (L % page != 0);
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < max_blocks; j += gridDim.x * blockDim.x)
+        order[(int64_t)b * row_stride + j] = j < N ? (j == 0 ? 0 : N - j) : -1;
+}
+
 using art::Layout;
 
 // ---------------------------------------------------------------- checks ----
@@ -155,7 +170,8 @@ art_status_t check_params(const art_params_t *p)
         return ART_ERR_PARAM;
     if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
         p->stages > 8 || p->compute_warps < 0 || p->compute_warps > art::kMaxComputeWarps || p->window < 0 ||
-        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64)
+        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64 ||
+        p->detector_off < 0 || p->detector_off > 1)
         return ART_ERR_PARAM;
     if (p->stages == 1 || (p->window > 0 && p->window < art::kMinWindow))
         return ART_ERR_PARAM;
@@ -169,21 +185,7 @@ art_status_t check_params(const art_params_t *p)
 
 // ------------------------------------------------------------- kernels ----
 
-using KernelFn = void (*)(KernelArgs, CUtensorMap, CUtensorMap);
-
-template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW>
-KernelFn kfn()
-{
-    return art::art_walk_kernel<T, D, PAGE, GMAX, ENGINE, NMW>;
-}
-
-template <typename T, int ENGINE, int GMAX, int NMW>
-KernelFn pick_dp(int d, int page)
-{
-    if (d == 64)
-        return page == 16 ? kfn<T, 64, 16, GMAX, ENGINE, NMW>() : kfn<T, 64, 64, GMAX, ENGINE, NMW>();
-    return page == 16 ? kfn<T, 128, 16, GMAX, ENGINE, NMW>() : kfn<T, 128, 64, GMAX, ENGINE, NMW>();
-}
+using art_walk::KernelFn;
 
 template <int ENGINE, int GMAX, int NMW>
 int merge_warps_dg(int d)
@@ -214,46 +216,18 @@ int gmax_for(int G, int engine)
     return G <= 1 ? 1 : (G <= 4 ? 4 : 8);
 }
 
-KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax, int nmw)
+KernelFn pick_kernel(int dtype, int engine, int d, int page, int gmax, int nmw, bool detector)
 {
-    if (dtype == ART_F32) {
-        if (gmax == 1) return pick_dp<float, art::kEngineCuda, 1, 1>(d, page);
-        if (gmax == 4) return pick_dp<float, art::kEngineCuda, 4, 1>(d, page);
-        return pick_dp<float, art::kEngineCuda, 8, 1>(d, page);
-    }
-    if (engine == art::kEngineMma) {
-        if (nmw == 4)
-            return gmax == 4 ? pick_dp<__nv_bfloat16, art::kEngineMma, 4, 4>(d, page)
-                             : pick_dp<__nv_bfloat16, art::kEngineMma, 8, 4>(d, page);
-        return gmax == 4 ? pick_dp<__nv_bfloat16, art::kEngineMma, 4, 1>(d, page)
-                         : pick_dp<__nv_bfloat16, art::kEngineMma, 8, 1>(d, page);
-    }
-    if (gmax == 1) return pick_dp<__nv_bfloat16, art::kEngineCuda, 1, 1>(d, page);
-    if (gmax == 4) return pick_dp<__nv_bfloat16, art::kEngineCuda, 4, 1>(d, page);
-    return pick_dp<__nv_bfloat16, art::kEngineCuda, 8, 1>(d, page);
-}
-
-// Two query tokens per walk (head dim 128): bf16 on the tensor-core engine,
-// fp32 on the CUDA-core engine.
-template <typename T, int ENGINE, int GMAX, int NMW>
-KernelFn pick_page_multi(int page)
-{
-    return page == 16 ? art::art_walk_kernel<T, 128, 16, GMAX, ENGINE, NMW, 2>
-                      : art::art_walk_kernel<T, 128, 64, GMAX, ENGINE, NMW, 2>;
+    if (dtype == ART_F32)
+        return art_walk::f32_cuda(gmax, d, page, detector);
+    if (engine == art::kEngineMma)
+        return art_walk::bf16_mma(gmax, nmw, d, page, detector);
+    return detector ? art_walk::bf16_cuda(gmax, d, page) : nullptr;
 }
 
 KernelFn pick_kernel_multi(int dtype, int engine, int page, int gmax, int nmw)
 {
-    if (dtype == ART_F32)
-        return gmax == 4 ? pick_page_multi<float, art::kEngineCuda, 4, 1>(page)
-                         : pick_page_multi<float, art::kEngineCuda, 8, 1>(page);
-    if (engine != art::kEngineMma)
-        return nullptr;
-    if (nmw == 4)
-        return gmax == 4 ? pick_page_multi<__nv_bfloat16, art::kEngineMma, 4, 4>(page)
-                         : pick_page_multi<__nv_bfloat16, art::kEngineMma, 8, 4>(page);
-    return gmax == 4 ? pick_page_multi<__nv_bfloat16, art::kEngineMma, 4, 1>(page)
-                     : pick_page_multi<__nv_bfloat16, art::kEngineMma, 8, 1>(page);
+    return art_walk::multi(dtype == ART_F32, engine, page, gmax, nmw);
 }
 
 // ------------------------------------------------------ device caches ----
@@ -510,8 +484,10 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     Shape s;
     if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
         return st;
+    if (nq > 1 && p->detector_off)
+        return ART_ERR_UNSUPPORTED;
     KernelFn fn = nq > 1 ? pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw)
-                         : pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw);
+                         : pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw, !p->detector_off);
     if (!fn)
         return ART_ERR_UNSUPPORTED;
     if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
@@ -674,7 +650,7 @@ art_status_t art_build_order_sink_recency(const art_tensor_t *seq_lens, int32_t 
     const int threads = 256;
     int gx = (mb + threads - 1) / threads;
     gx = gx > 64 ? 64 : gx;
-    art::art_build_order_kernel<<<dim3(gx, (unsigned)B), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    art_build_order_kernel<<<dim3(gx, (unsigned)B), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         static_cast<const int32_t *>(seq_lens->data), (int)B, page, static_cast<int32_t *>(block_order->data),
         block_order->stride[0], mb);
     if (cudaGetLastError() != cudaSuccess)

@@ -941,7 +941,13 @@ __device__ __forceinline__ void merge_barrier2(int nthreads)
 // reaching the same decision.  A stop inside a batch replays the batch up to
 // the stop from a snapshot, so the stop and the output are those of a
 // strictly sequential walk.
-template <int D, int GMAX, int ENGINE, int NMW>
+//
+// DET = false builds the same walk without the detector: the blocks are folded
+// exactly as above (the same batches, shares and arithmetic, so the output
+// equals the eps = 0 walk's bit for bit), but no statistic is formed, no
+// patience rule runs and the walk never stops early.  It exists as the timing
+// reference for the detector's cost.
+template <int D, int GMAX, int ENGINE, int NMW, bool DET = true>
 __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, int N, int mw)
 {
     using MS = MergeShape<D, GMAX, ENGINE, NMW>;
@@ -1020,12 +1026,15 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 continue;
 #pragma unroll
             for (int q = 0; q < VP; ++q) {
-                const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
+                // o += beta (u - o) as one fused step (one rounding); written
+                // as such so that no instantiation fuses it differently
+                const uint64_t df = sub2(uv[ii][q], o[ii][q]);
                 if (sums) {
+                    const uint64_t dl = mul2(bp[ii], df);
                     sd = fma2(o[ii][q], dl, sd);
                     se = fma2(dl, dl, se);
                 }
-                o[ii][q] = add2(o[ii][q], dl);
+                o[ii][q] = fma2(bp[ii], df, o[ii][q]);
             }
         }
         if (sums) {
@@ -1149,7 +1158,9 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 #pragma unroll
                 for (int off = GMAX; off < 32; off <<= 1)
                     Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, off));
-                const float w = (mk == -CUDART_INF_F) ? 0.f : lk * ex2_approx(mk - Mb);
+                // (explicitly rounded products: the compiler may not fuse them into a
+                // later add, so every instantiation folds with the same arithmetic)
+                const float w = (mk == -CUDART_INF_F) ? 0.f : __fmul_rn(lk, ex2_approx(mk - Mb));
                 float S = w;
 #pragma unroll
                 for (int off = GMAX; off < 32; off <<= 1) {
@@ -1157,8 +1168,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                     if (lane >= off)
                         S += t;
                 }
-                const float Lam = ((Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb)) + S;
-                beta = Lam > 0.f ? w * rcp_approx(Lam) : 0.f;
+                const float Lam = ((Mx == -CUDART_INF_F) ? 0.f : __fmul_rn(Lm, ex2_approx(Mx - Mb))) + S;
+                beta = Lam > 0.f ? __fmul_rn(w, rcp_approx(Lam)) : 0.f;
                 Lm = __shfl_sync(0xffffffffu, Lam, (nb - 1) * GMAX + gl);
             } else {  // two rows: entry hh of a lane is block kl + hh KH
                 float mk[NH], lk[NH];
@@ -1183,7 +1194,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 float w[NH], S[NH];
 #pragma unroll
                 for (int hh = 0; hh < NH; ++hh) {
-                    w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : lk[hh] * ex2_approx(mk[hh] - Mb);
+                    w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : __fmul_rn(lk[hh], ex2_approx(mk[hh] - Mb));
                     S[hh] = w[hh];
                 }
 #pragma unroll
@@ -1196,12 +1207,12 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                     }
                 if constexpr (NH > 1)  // the second row follows the whole first row
                     S[1] += __shfl_sync(0xffffffffu, S[0], (KH - 1) * GMAX + gl);
-                const float base = (Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb);
+                const float base = (Mx == -CUDART_INF_F) ? 0.f : __fmul_rn(Lm, ex2_approx(Mx - Mb));
                 float Lam[NH], bh[NH];
 #pragma unroll
                 for (int hh = 0; hh < NH; ++hh) {
                     Lam[hh] = base + S[hh];
-                    bh[hh] = Lam[hh] > 0.f ? w[hh] * rcp_approx(Lam[hh]) : 0.f;
+                    bh[hh] = Lam[hh] > 0.f ? __fmul_rn(w[hh], rcp_approx(Lam[hh])) : 0.f;
                 }
                 beta = bh[0];
                 beta_hi = bh[NH - 1];
@@ -1209,17 +1220,41 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 Lm = __shfl_sync(0xffffffffu, Llast, ((nb - 1) % KH) * GMAX + gl);
             }
             Mx = Mb;
-            // 3. ||o||^2 before the batch, then fold the batch into this warp's slice
-            uint64_t n2 = 0ull;
+            if constexpr (DET) {
+                // 3. ||o||^2 before the batch, then fold the batch into this warp's slice
+                uint64_t n2 = 0ull;
 #pragma unroll
-            for (int i = 0; i < NVW; ++i)
+                for (int i = 0; i < NVW; ++i)
 #pragma unroll
-                for (int q = 0; q < VP; ++q) {
-                    o0[i][q] = o[i][q];
-                    n2 = fma2(o[i][q], o[i][q], n2);
-                }
-            n0part = lo2(n2) + hi2(n2);
-            fold_batch(s0, nb - 1, beta, beta_hi, v, true);
+                    for (int q = 0; q < VP; ++q) {
+                        o0[i][q] = o[i][q];
+                        n2 = fma2(o[i][q], o[i][q], n2);
+                    }
+                n0part = lo2(n2) + hi2(n2);
+            }
+            fold_batch(s0, nb - 1, beta, beta_hi, v, DET);
+        }
+        if constexpr (!DET) {
+            // no detector: the merge warps agreed on the batch (or the failure)
+            // before the fold; they meet once more so that no warp still reads
+            // the batch's slots when they are handed back to the producers
+            if (local_fail) {
+                failed = true;
+                break;
+            }
+            if constexpr (NM > 1)
+                merge_barrier(NM * 32);
+            else
+                __syncwarp();
+            if (mw == 0 && lane == 0)
+                st_relaxed_cluster_u32(ctrl_cl, (uint32_t)(j0 + nb));
+            j0 += nb;
+            s0 += nb;
+            if (s0 >= a.R) {
+                s0 -= a.R;
+                ph0 ^= 1u;
+            }
+            continue;
         }
         // 4. lane 2k+q (and 2k+q+16): sum over the warp of quantity q of batch block k
         reduce_scatter16(v, lane);
@@ -1452,12 +1487,14 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                 continue;  // padding rows: never written (see merge_role)
 #pragma unroll
             for (int q = 0; q < VP; ++q) {
-                const uint64_t dl = mul2(bp[ii], sub2(uv[ii][q], o[ii][q]));
+                // o += beta (u - o) as one fused step, as in merge_role
+                const uint64_t df = sub2(uv[ii][q], o[ii][q]);
                 if (sums) {
+                    const uint64_t dl = mul2(bp[ii], df);
                     sd[ii] = fma2(o[ii][q], dl, sd[ii]);
                     se[ii] = fma2(dl, dl, se[ii]);
                 }
-                o[ii][q] = add2(o[ii][q], dl);
+                o[ii][q] = fma2(bp[ii], df, o[ii][q]);
             }
         }
         if (sums) {
@@ -1591,7 +1628,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
             float w[NH], S[NH];
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) {
-                w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : lk[hh] * ex2_approx(mk[hh] - Mb);
+                w[hh] = (mk[hh] == -CUDART_INF_F) ? 0.f : __fmul_rn(lk[hh], ex2_approx(mk[hh] - Mb));
                 S[hh] = w[hh];
             }
 #pragma unroll
@@ -1610,13 +1647,13 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
                 if (hh + 1 < NH)
                     carry = __shfl_sync(0xffffffffu, S[hh], (KH - 1) * GMAX + gl);
             }
-            const float base = (Mx == -CUDART_INF_F) ? 0.f : Lm * ex2_approx(Mx - Mb);
+            const float base = (Mx == -CUDART_INF_F) ? 0.f : __fmul_rn(Lm, ex2_approx(Mx - Mb));
             const bool frozen = tok_gl < NQ && ((done >> tok_gl) & 1u);
             float Lam[NH];
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) {
                 Lam[hh] = base + S[hh];
-                bh[hh] = (Lam[hh] > 0.f && !frozen) ? w[hh] * rcp_approx(Lam[hh]) : 0.f;
+                bh[hh] = (Lam[hh] > 0.f && !frozen) ? __fmul_rn(w[hh], rcp_approx(Lam[hh])) : 0.f;
             }
             const int hl = (nb - 1) / KH;  // row of the batch's last block
             float Llast = Lam[0];
@@ -1797,7 +1834,8 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
 // ---- kernel ------------------------------------------------------------------------
 
 // NQ: query tokens sharing the walk (1: merge_role, else merge_role_multi).
-template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW, int NQ = 1>
+// DET: false for the single-query walk without the detector (see merge_role).
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW, int NQ = 1, bool DET = true>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv)
@@ -1873,7 +1911,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         else if (warp <= NM) {
             if (rank == 0) {
                 if constexpr (NQ == 1)
-                    merge_role<D, GMAX, ENGINE, NMW>(a, sh, b, h, N, warp - 1);
+                    merge_role<D, GMAX, ENGINE, NMW, DET>(a, sh, b, h, N, warp - 1);
                 else
                     merge_role_multi<D, GMAX, ENGINE, NMW, NQ>(a, sh, b, h, N, warp - 1);
             }
@@ -1901,19 +1939,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     cluster_sync();  // remote stores into the leader are complete
     if (rank == 0 && threadIdx.x == 0 && a.blocks_fetched)
         a.blocks_fetched[unit] = (int32_t)sh.fetched[0];
-}
-
-// Default walk order: [0, N-1, N-2, ..., 1], -1 beyond N.
-__global__ void art_build_order_kernel(const int32_t *seq_lens, int B, int page, int32_t *order, int64_t row_stride,
-                                       int max_blocks)
-{
-    const int b = blockIdx.y;
-    if (b >= B)
-        return;
-    const int L = seq_lens[b];
-    const int N = L <= 0 ? 0 : L / page + (L % page != 0);
-    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < max_blocks; j += gridDim.x * blockDim.x)
-        order[(int64_t)b * row_stride + j] = j < N ? (j == 0 ? 0 : N - j) : -1;
 }
 
 }  // namespace art

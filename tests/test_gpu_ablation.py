@@ -134,3 +134,56 @@ def test_length_near_int32_max_reported(cuda_lib):
     assert order[2, 0].item() == 0 and (order[2, 1:] > 0).all()
     ok = parity.subset_sequences(w, [0, 1])
     parity.check(ok, out[:2], stop[:2])
+
+
+# ----------------------------------------------------------- detector off ----
+
+@pytest.mark.parametrize("case", ["llama8b_b8", "qwen7b_b4", "tiny_fp32", "many_g8", "many_g4"])
+def test_detector_off_equals_eps0(cuda_lib, case):
+    """The walk built without the detector (no statistic, no patience, no
+    early stop) gives the eps = 0 walk's stops and output bit for bit, in the
+    same launch shape; and both equal the oracle's full softmax attention."""
+    from kv_cache_early_art_b200.workloads import make_workload
+    if case == "many_g8":
+        w = make_custom(B=40, Hq=28, Hkv=4, d=128, page=64, dtype="bf16",
+                        seq_lens=[64 * (10 + b) + 7 * b for b in range(40)], seed=61)
+    elif case == "many_g4":
+        w = make_custom(B=48, Hq=16, Hkv=4, d=128, page=64, dtype="bf16",
+                        seq_lens=[64 * (5 + 2 * b) + b for b in range(48)], seed=62)
+    else:
+        w = make_workload(case)
+    g = w.to("cuda")
+    zero = torch.zeros(w.B, dtype=torch.float32, device="cuda")
+    kw = dict(eps_m_per_seq=zero, eps_d_per_seq=zero, P_per_seq=g.P, min_blocks_per_seq=g.min_blocks)
+    out0, stop0, info0 = cuda_lib.art_decode_attention_ex(g.q, g.k_cache, g.v_cache, g.page_table, None, g.seq_lens,
+                                                          want_info=True, **kw)
+    fetched = torch.zeros(w.B * w.Hkv, dtype=torch.int32, device="cuda")
+    out1, stop1, info1 = cuda_lib.art_decode_attention_ex(g.q, g.k_cache, g.v_cache, g.page_table, None, g.seq_lens,
+                                                          detector_off=1, blocks_fetched=fetched, want_info=True,
+                                                          **kw)
+    torch.cuda.synchronize()
+    assert info0 == info1
+    N = w.n_blocks().numpy()[:, None]
+    assert (stop1.cpu().numpy() == N).all() and (fetched.view(w.B, w.Hkv).cpu().numpy() == N).all()
+    assert torch.equal(stop0, stop1) and torch.equal(out0, out1)
+    wc = w.to("cpu")
+    wc.eps_m, wc.eps_d = torch.zeros(w.B), torch.zeros(w.B)
+    parity.check(wc, out1, stop1)
+
+
+def test_detector_off_where_not_built(cuda_lib):
+    """Shapes without a detector-off build, and the shared walk, refuse it."""
+    w = make_custom(B=2, Hq=8, Hkv=2, d=128, page=64, dtype="bf16", seq_lens=[300, 200], seed=63).to("cuda")
+    with pytest.raises(cuda_lib.ArtError) as e:
+        cuda_lib.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
+                                         detector_off=1, engine=1)
+    assert e.value.status == -4
+    qm = torch.stack([w.q, w.q], dim=1)
+    with pytest.raises(cuda_lib.ArtError) as e:
+        cuda_lib.art_decode_attention_multi(qm, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
+                                            detector_off=1)
+    assert e.value.status == -4
+    with pytest.raises(cuda_lib.ArtError) as e:
+        cuda_lib.art_decode_attention_ex(w.q, w.k_cache, w.v_cache, w.page_table, None, w.seq_lens,
+                                         detector_off=2)
+    assert e.value.status == -5
