@@ -113,9 +113,13 @@ typedef struct {
     int32_t threads;       /* threads per CTA                                             */
     int32_t stages;        /* K/V pages buffered per CTA                                  */
     int32_t compute_warps; /* warps turning pages into block states, per CTA              */
-    int32_t window;        /* blocks staged ahead of the merged prefix (state ring slots)  */
+    int32_t window;        /* blocks fetched ahead of the merged prefix (the bound on      */
+                           /* pages read past the stop)                                    */
     int32_t smem_bytes;    /* dynamic shared memory per CTA                               */
     int32_t prefetch;      /* further blocks pulled into L2 ahead of the staged ones      */
+    int32_t merge_cta;     /* 1: the cluster's first CTA only merges                      */
+    int32_t ring_slots;    /* block states the merging CTA holds (= window, or fewer with */
+                           /* merge_cta: then a finished state waits for a free slot)     */
 } art_launch_info_t;
 
 typedef struct {
@@ -134,7 +138,10 @@ typedef struct {
     int32_t cluster_size;          /* 0 auto, else 1..16 CTAs per unit                      */
     int32_t stages;                /* 0 auto, else 2..8 (a multiple of compute_warps)       */
     int32_t compute_warps;         /* 0 auto, else 1..6                                     */
-    int32_t window;                /* 0 auto, else 8..64 blocks of speculation              */
+    int32_t window;                /* 0 auto, else 8..128 blocks fetched ahead of the       */
+                                   /* merged prefix (speculation; pages read past the stop  */
+                                   /* stay below it).  Without merge_cta it is also the     */
+                                   /* state ring's size, which must fit in shared memory    */
     int64_t timeout_ns;            /* 0 = 2 s; bound on every device-side wait              */
     int32_t debug_flags;           /* 0; bit 0 makes the stop decision wait on a barrier    */
                                    /* nothing arrives on (exercises the bounded wait)       */
@@ -154,6 +161,17 @@ typedef struct {
                                    /* at most 4 query heads per kv head; other cases return */
                                    /* ART_ERR_UNSUPPORTED, as does art_decode_attention_multi*/
                                    /* with n_queries = 2.                                   */
+    int32_t merge_cta;             /* 0 auto; 1: the first CTA of each cluster only merges  */
+                                   /* (its whole shared memory holds the block states, so   */
+                                   /* the window can reach 64; its warps fold in parallel   */
+                                   /* and one warp decides a batch behind them) while the   */
+                                   /* others fetch and compute; -1 never.  Auto picks it    */
+                                   /* for fewer units than SMs with clusters of 4 or more   */
+                                   /* CTAs.  Built for BF16 caches on the tensor-core       */
+                                   /* engine, d = 128, 64-token pages, single-query walks;  */
+                                   /* 1 elsewhere returns ART_ERR_UNSUPPORTED, and with     */
+                                   /* cluster_size 1 ART_ERR_PARAM.  Stops and outputs are  */
+                                   /* the sequential rule's, as with every launch shape.    */
 } art_params_t;
 
 /*

@@ -40,7 +40,8 @@ class ArtTensor(ctypes.Structure):
 
 class ArtLaunchInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("engine", "cluster_size", "grid", "threads", "stages",
-                                               "compute_warps", "window", "smem_bytes", "prefetch")]
+                                               "compute_warps", "window", "smem_bytes", "prefetch", "merge_cta",
+                                               "ring_slots")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -57,7 +58,7 @@ class ArtParams(ctypes.Structure):
         ("engine", ctypes.c_int32), ("cluster_size", ctypes.c_int32), ("stages", ctypes.c_int32),
         ("compute_warps", ctypes.c_int32), ("window", ctypes.c_int32), ("timeout_ns", ctypes.c_int64),
         ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo)), ("prefetch", ctypes.c_int32),
-        ("detector_off", ctypes.c_int32)]
+        ("detector_off", ctypes.c_int32), ("merge_cta", ctypes.c_int32)]
 
 
 _P = ctypes.POINTER
@@ -147,7 +148,8 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
 
 def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P, min_blocks,
             sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status,
-            engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch, detector_off=0):
+            engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch, detector_off=0,
+            merge_cta=0):
     """Fill art_params_t (argument marshalling only); returns (params, info)."""
     per = [eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status]
     _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, *per)
@@ -172,6 +174,7 @@ def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_bl
     p.debug_flags = int(debug_flags)
     p.prefetch = int(prefetch)
     p.detector_off = int(detector_off)
+    p.merge_cta = int(merge_cta)
     info = ArtLaunchInfo()
     p.info = ctypes.pointer(info)
     return p, info
@@ -181,8 +184,8 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
                             P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                             P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                             engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                            debug_flags=0, prefetch=0, detector_off=0, out=None, stop_block=None, stream=None,
-                            want_info=False):
+                            debug_flags=0, prefetch=0, detector_off=0, merge_cta=0, out=None, stop_block=None,
+                            stream=None, want_info=False):
     """art_decode_attention_ex in art.h.  Per-sequence arrays are device
     tensors of length B (float32 thresholds, int32 P / min_blocks).
     Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
@@ -194,7 +197,7 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch, detector_off)
+                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta)
     st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
     _check(st, "art_decode_attention_ex")
     if want_info:
@@ -206,8 +209,8 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
                                P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                                P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                                engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                               debug_flags=0, prefetch=0, detector_off=0, out=None, stop_block=None, stream=None,
-                               want_info=False):
+                               debug_flags=0, prefetch=0, detector_off=0, merge_cta=0, out=None, stop_block=None,
+                               stream=None, want_info=False):
     """art_decode_attention_multi in art.h: q [B, T, Hq, d], T query tokens
     per sequence sharing one walk.  Returns (out [B, T, Hq, d],
     stop_block [B, T, Hkv]) or those plus the launch info dict."""
@@ -219,7 +222,7 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch, detector_off)
+                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta)
     st = _lib.art_decode_attention_multi(ctypes.byref(p), int(T), _stream(stream))
     _check(st, "art_decode_attention_multi")
     if want_info:

@@ -15,7 +15,7 @@ LIB = os.path.join(HERE, "libart.so")
 # one translation unit per group of walk instantiations, so that they compile in parallel
 SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu", "art_order.cu", "art_walk_f32.cu", "art_walk_bf16.cu",
                                            "art_walk_mma.cu", "art_walk_multi.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh", "art_host.h", "art_walk.h")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh", "art_host.h", "art_walk.h", "art_walk_dl.cuh")] + [
     os.path.join(ROOT, "include", "art.h")]
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@
 #include "art_host.h"
 #include "art_kernels.cuh"
 #include "art_walk.h"
+#include "art_walk_dl.cuh"
 
 namespace {
 
@@ -170,8 +171,8 @@ art_status_t check_params(const art_params_t *p)
         return ART_ERR_PARAM;
     if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
         p->stages > 8 || p->compute_warps < 0 || p->compute_warps > art::kMaxComputeWarps || p->window < 0 ||
-        p->window > 64 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64 ||
-        p->detector_off < 0 || p->detector_off > 1)
+        p->window > 128 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64 ||
+        p->detector_off < 0 || p->detector_off > 1 || p->merge_cta < -1 || p->merge_cta > 1)
         return ART_ERR_PARAM;
     if (p->stages == 1 || (p->window > 0 && p->window < art::kMinWindow))
         return ART_ERR_PARAM;
@@ -318,7 +319,32 @@ art_status_t make_cache_map(CUtensorMap *map, const art_tensor_t *c, int dtype, 
 
 struct Shape {
     int engine, gmax, nmw, S, NW, R, C, PF, smem, threads;
+    int RF = 0;              // window (blocks fetched ahead of the merged prefix); R = ring slots
+    int dl = 0;              // 1: dedicated merge CTA (art_walk_dl_kernel)
+    KernelFn fn = nullptr;   // set by the dedicated-merge choice
 };
+
+// clusters of C CTAs of fn (threads, smem) that can be resident at once (0 if none)
+int resident_clusters(KernelFn fn, int threads, int smem, int units, int C)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(units * C);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, (void *)fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return nclusters;
+}
 
 int smem_bytes(const Shape &s, const Problem &pr)
 {
@@ -392,6 +418,7 @@ art_status_t choose_shape(const art_params_t *p, const Problem &pr, const Device
         s.NW = NW;
         s.S = S;
         s.R = p->window ? p->window : cand[i][2];
+        s.RF = s.R;
         s.threads = 32 * (1 + merge_warps(s.engine, pr.d, s.gmax, s.nmw) + NW);
         s.smem = smem_bytes(s, pr);
         if (s.smem <= di.smem_optin) {
@@ -414,26 +441,7 @@ art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const Device
         return ART_ERR_LAUNCH;
     per_sm = per_sm < 1 ? 1 : per_sm;
     const int slots = di.sms * per_sm;
-    // clusters of C CTAs that can be resident at once (0 if none)
-    auto resident = [&](int C) -> int {
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(units * C);
-        cfg.blockDim = dim3(s->threads);
-        cfg.dynamicSmemBytes = s->smem;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, (void *)fn, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            return 0;
-        }
-        return nclusters;
-    };
+    auto resident = [&](int C) -> int { return resident_clusters(fn, s->threads, s->smem, units, C); };
     int C = 1;
     if (units < slots) {
         // one wave: the largest cluster size whose clusters all fit at once
@@ -465,6 +473,103 @@ art_status_t pick_cluster(KernelFn fn, Shape *s, const Problem &pr, const Device
     return ART_OK;
 }
 
+// Dedicated merge CTA (art_walk_dl_kernel): rank 0 of each cluster holds the
+// state ring in all of its shared memory and only merges; the other ranks
+// fetch and compute.  Chosen automatically for fewer units than SMs when at
+// least four CTAs per unit fit at once (the merge CTA costs one fetching CTA,
+// so small clusters keep art_walk_kernel); merge_cta = 1 asks for it.
+// *chosen stays false when art_walk_kernel should run instead.
+art_status_t choose_dl(const art_params_t *p, const Problem &pr, const DeviceInfo &di, Shape *out, bool *chosen)
+{
+    *chosen = false;
+    const bool forced = p->merge_cta == 1;
+    const int engine = p->engine ? p->engine : (pr.dtype == ART_BF16 ? art::kEngineMma : art::kEngineCuda);
+    if (engine != art::kEngineMma || pr.dtype != ART_BF16 || pr.d != 128 || pr.page != 64)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    const int units = pr.B * pr.Hkv;
+    if (!forced && units >= di.sms)
+        return ART_OK;
+    if (p->cluster_size == 1)
+        return forced ? ART_ERR_PARAM : ART_OK;
+    if (p->compute_warps && p->stages && p->stages % p->compute_warps != 0)
+        return ART_ERR_PARAM;
+    Shape s;
+    s.engine = art::kEngineMma;
+    s.gmax = gmax_for(pr.G, s.engine);
+    s.nmw = s.gmax;  // one fold warp per 16 output floats of a lane: 4 or 8
+    s.PF = p->prefetch > 0 ? p->prefetch : 0;
+    s.dl = 1;
+    const int es = (int)elem_size(pr.dtype);
+    const int limit = di.smem_optin - 1024;  // slack to align the base to 1024 bytes
+    // the merge CTA's ring: as deep as fits, in whole merge batches, at most
+    // 64 slots and at most the window
+    const int cap = p->window && p->window < 64 ? p->window : 64;
+    int R = cap;
+    for (; R > art::kMinWindow; R -= R % 8 ? R % 8 : 8)
+        if ((int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total <= limit)
+            break;
+    if ((int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total > limit)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    s.R = R;
+    // the fetching CTAs: (compute warps, stages), deepest first
+    static const int cand[][2] = {{6, 6}, {3, 6}, {5, 5}, {4, 4}, {2, 4}, {2, 2}, {1, 2}};
+    bool fit = false;
+    for (const auto &c : cand) {
+        int NW = p->compute_warps ? p->compute_warps : c[0];
+        int S = p->stages ? p->stages : c[1];
+        if (p->stages && !p->compute_warps) {
+            while (S % NW != 0)
+                --NW;
+        } else if (!p->stages) {
+            S = NW * ((S + NW - 1) / NW);
+            if (S > 8)
+                S = NW * (8 / NW);
+        }
+        if ((int)art::make_dl_layout(S, R, pr.page, pr.d, es, s.gmax, 0).total <= limit) {
+            s.NW = NW;
+            s.S = S;
+            fit = true;
+            break;
+        }
+    }
+    if (!fit)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    const int lead = (int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total;
+    const int work = (int)art::make_dl_layout(s.S, R, pr.page, pr.d, es, s.gmax, 0).total;
+    s.smem = (lead > work ? lead : work) + 1024;
+    s.threads = 32 * (2 + s.nmw > 1 + s.NW ? 2 + s.nmw : 1 + s.NW);
+    s.fn = art_walk::bf16_mma_dl(s.gmax, pr.d, pr.page, !p->detector_off);
+    if (!s.fn)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    art_status_t st = prepare_kernel(s.fn, s.smem);
+    if (st != ART_OK)
+        return st;
+    int C = p->cluster_size;
+    if (!C) {
+        // the largest cluster whose clusters are all resident at once
+        C = di.sms / units;
+        C = C > 16 ? 16 : C;
+        for (; C > 2; --C)
+            if (resident_clusters(s.fn, s.threads, s.smem, units, C) >= units)
+                break;
+        if (C < 2 || resident_clusters(s.fn, s.threads, s.smem, units, C) < 1)
+            return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+        if (!forced && C < 4)
+            return ART_OK;
+    }
+    s.C = C;
+    // the window reaches past the ring by the pages the fetching CTAs can hold
+    // in their stages: those are fetched and computed while the merge still
+    // holds every slot, and their states wait for a slot (slot_gate)
+    s.RF = p->window ? p->window : s.R + (C - 1) * s.S;
+    s.RF = s.RF > 128 ? 128 : s.RF;
+    if (s.RF < s.R)
+        s.RF = s.R;
+    *out = s;
+    *chosen = true;
+    return ART_OK;
+}
+
 // tokens_dim: q and out are [B, T, Hq, d] and stop_block [B, T, Hkv] (T = nq)
 art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool tokens_dim = false)
 {
@@ -481,17 +586,27 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     DeviceInfo di;
     if ((st = device_info(&di)) != ART_OK)
         return st;
-    Shape s;
-    if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
-        return st;
     if (nq > 1 && p->detector_off)
         return ART_ERR_UNSUPPORTED;
-    KernelFn fn = nq > 1 ? pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw)
-                         : pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw, !p->detector_off);
-    if (!fn)
+    if (nq > 1 && p->merge_cta == 1)
         return ART_ERR_UNSUPPORTED;
-    if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
+    Shape s;
+    bool dl = false;
+    if (nq == 1 && p->merge_cta != -1 && (st = choose_dl(p, pr, di, &s, &dl)) != ART_OK)
         return st;
+    KernelFn fn = nullptr;
+    if (dl) {
+        fn = s.fn;
+    } else {
+        if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
+            return st;
+        fn = nq > 1 ? pick_kernel_multi(pr.dtype, s.engine, pr.page, s.gmax, s.nmw)
+                    : pick_kernel(pr.dtype, s.engine, pr.d, pr.page, s.gmax, s.nmw, !p->detector_off);
+        if (!fn)
+            return ART_ERR_UNSUPPORTED;
+        if ((st = prepare_kernel(fn, s.smem)) != ART_OK)
+            return st;
+    }
 
     KernelArgs ka;
     std::memset(&ka, 0, sizeof ka);
@@ -537,12 +652,13 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     ka.out_st = pr.out_st;
     ka.stop_st = pr.stop_st;
 
-    if ((st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
+    if (!dl && (st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
         return st;
     ka.C = s.C;
     ka.S = s.S;
     ka.NW = s.NW;
     ka.R = s.R;
+    ka.RF = s.RF;
     ka.PF = s.PF;
 
     CUtensorMap tmk, tmv;
@@ -572,9 +688,11 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
         p->info->threads = s.threads;
         p->info->stages = s.S;
         p->info->compute_warps = s.NW;
-        p->info->window = s.R;
+        p->info->window = s.RF;
+        p->info->ring_slots = s.R;
         p->info->prefetch = s.PF;
         p->info->smem_bytes = s.smem;
+        p->info->merge_cta = s.dl;
     }
     if (cudaLaunchKernelEx(&cfg, fn, ka, tmk, tmv) != cudaSuccess) {
         cudaGetLastError();

@@ -68,7 +68,9 @@ struct KernelArgs {
     int32_t *blocks_fetched;
     int32_t *device_status;
     int32_t B, Hq, Hkv, G, num_pages, max_blocks;
-    int32_t C, S, NW, R;                // cluster size, stages, compute warps, window
+    int32_t C, S, NW, R;                // cluster size, stages, compute warps, state-ring slots
+    int32_t RF;                         // window: blocks fetched ahead of the merged prefix (>= R; above R
+                                        // a finished block state waits for its slot)
     int32_t PF;                         // pages pulled into L2 ahead of the staged loads
     int64_t timeout_ns;
     int32_t debug_flags;
@@ -251,24 +253,32 @@ struct Shared {
     float *pbuf;          // per compute warp [PAGE][GMAX] (CUDA-core engine)
     float *red;           // merge-warp exchange
     uint32_t *stage_j, *stage_nv;
-    uint32_t bar0;        // shared address of full_k[0]
+    // shared addresses of the mbarrier arrays
+    uint32_t bar_full_k, bar_full_v, bar_empty, bar_ready, bar_never;
+    // this CTA's shared addresses at which the leader (rank 0) keeps its state
+    // ring and the ring's ready barriers (mapped to rank 0 with mapa)
+    uint32_t ring_leader, ready_leader;
     volatile uint32_t *ctrl, *fetched, *abort;
     Layout L;
-    __device__ uint32_t full_k(int s) const { return bar0 + 8u * s; }
-    __device__ uint32_t full_v(int s, int S) const { return bar0 + 8u * (S + s); }
-    __device__ uint32_t empty(int s, int S) const { return bar0 + 8u * (2 * S + s); }
-    __device__ uint32_t ready(int r, int S) const { return bar0 + 8u * (3 * S + r); }
-    __device__ uint32_t never(int S, int R) const { return bar0 + 8u * (3 * S + R); }
+    __device__ uint32_t full_k(int s) const { return bar_full_k + 8u * s; }
+    __device__ uint32_t full_v(int s) const { return bar_full_v + 8u * s; }
+    __device__ uint32_t empty(int s) const { return bar_empty + 8u * s; }
+    __device__ uint32_t ready(int r) const { return bar_ready + 8u * r; }
+    __device__ uint32_t never() const { return bar_never; }
 };
 
 // ---- producer ----------------------------------------------------------------
 
-template <typename T, int D, int PAGE, int ENGINE>
+// rank, C: this CTA's place among the CTAs that fetch for the unit and their
+// number (steps j = rank, rank + C, ... are this CTA's).  kAcquire: read the
+// merged progress with acquire semantics (needed where the warp that publishes
+// it is not the one that read the freed slots).
+template <typename T, int D, int PAGE, int ENGINE, bool kAcquire = false>
 __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUtensorMap *tmk, const CUtensorMap *tmv,
-                              int b, int h, int N, int Lseq, uint32_t rank, int first_lb, int first_pp)
+                              int b, int h, int N, int Lseq, uint32_t rank, int C, int first_lb, int first_pp)
 {
     const int lane = threadIdx.x & 31;
-    const int S = a.S, R = a.R, C = a.C;
+    const int S = a.S, R = a.RF;
     const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
     const int32_t *bo = a.block_order ? a.block_order + (int64_t)b * a.bo_sb : nullptr;
     const int32_t *pt = a.page_table + (int64_t)b * a.pt_sb;
@@ -292,7 +302,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         const int s = (int)(i % (uint32_t)S);
         if (i < (uint32_t)S)
             return true;
-        return warp_wait<false>(sh.empty(s, S), ((i / S) - 1) & 1u, sh.abort, a.timeout_ns, a.device_status);
+        return warp_wait<false>(sh.empty(s), ((i / S) - 1) & 1u, sh.abort, a.timeout_ns, a.device_status);
     };
 
     for (int k = 0;; ++k) {
@@ -322,7 +332,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         if (lane == 0 && ((uint32_t)j >= ctrl_cache + (uint32_t)R || (k & 3) == 0)) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const uint32_t c = ld_relaxed_cluster_u32(ctrl_cl);
+                const uint32_t c = kAcquire ? ld_acquire_cluster_u32(ctrl_cl) : ld_relaxed_cluster_u32(ctrl_cl);
                 if (c & kStopBit) { go = 0; break; }
                 ctrl_cache = c;
                 if ((uint32_t)j < c + (uint32_t)R) break;
@@ -354,7 +364,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
                 // pass the fault down the pipeline: the merge reports it
                 sh.stage_nv[s] = 0xFFFFFFFFu;
                 mbar_arrive(sh.full_k(s));
-                mbar_arrive(sh.full_v(s, S));
+                mbar_arrive(sh.full_v(s));
                 record_error(a.device_status, kErrBadIndex);
             } else {
                 const int nv = min(PAGE, Lseq - lb * PAGE);
@@ -369,13 +379,13 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
                 } else {
                     tma_load_4d(kdst, tmk, 0, 0, h, pp, sh.full_k(s));
                 }
-                mbar_arrive_expect_tx(sh.full_v(s, S), sh.L.tile_bytes);
+                mbar_arrive_expect_tx(sh.full_v(s), sh.L.tile_bytes);
                 if constexpr (ENGINE == kEngineMma) {
 #pragma unroll
                     for (int sb = 0; sb < D / 64; ++sb)
-                        tma_load_4d(vdst + sb * PAGE * 128, tmv, sb * 64, 0, h, pp, sh.full_v(s, S));
+                        tma_load_4d(vdst + sb * PAGE * 128, tmv, sb * 64, 0, h, pp, sh.full_v(s));
                 } else {
-                    tma_load_4d(vdst, tmv, 0, 0, h, pp, sh.full_v(s, S));
+                    tma_load_4d(vdst, tmv, 0, 0, h, pp, sh.full_v(s));
                 }
             }
         }
@@ -445,7 +455,7 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
             if (kused >> s & 1u)
                 warp_wait<false>(sh.full_k(s), kphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
             if (vused >> s & 1u)
-                warp_wait<false>(sh.full_v(s, S), vphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
+                warp_wait<false>(sh.full_v(s), vphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
         }
     }
     if (lane == 0)
@@ -461,7 +471,52 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
 struct SlotRef {
     uint32_t base;   // cluster address of the slot
     uint32_t ready;  // cluster address of its ready barrier
+    uint32_t need;   // the slot is free once the merged count reaches this (0: it is free)
+    uint32_t ctrl;   // cluster address of the merged count
 };
+
+// Wait (whole warp, bounded) until the slot a finished block state goes to
+// is free: the block R places earlier in the walk has been merged.  Needed
+// only where the window reaches past the state ring.  Returns 1 to push, 0 to
+// drop the state (the walk has stopped, or failed, before it), -1 on timeout
+// or abort.  cache holds the last merged count this warp read.
+static __device__ __noinline__ int slot_gate(const KernelArgs &a, const Shared &sh, const SlotRef &sr, uint32_t &cache)
+{
+    int r = 0;
+    if ((threadIdx.x & 31) == 0) {
+        uint64_t t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+            if (cache & kStopBit) {
+                r = 0;
+                break;
+            }
+            if (cache >= sr.need) {
+                r = 1;
+                break;
+            }
+            cache = ld_acquire_cluster_u32(sr.ctrl);
+            if ((it & 15u) == 15u) {
+                const uint64_t now = global_timer_ns();
+                if (t0 == 0)
+                    t0 = now;
+                if (*sh.abort) {
+                    r = -1;
+                    break;
+                }
+                if ((int64_t)(now - t0) > a.timeout_ns) {
+                    *sh.abort = 1u;
+                    record_error(a.device_status, kErrTimeout);
+                    r = -1;
+                    break;
+                }
+            }
+        }
+    }
+    r = __shfl_sync(0xffffffffu, r, 0);
+    cache = __shfl_sync(0xffffffffu, cache, 0);
+    __syncwarp();  // the lanes' slot writes come after lane 0's acquire
+    return r;
+}
 
 // Bytes one block state occupies in a slot: flag word, m and l per head,
 // and the normalised output u (all GMAX heads for the tensor-core layout,
@@ -504,7 +559,7 @@ struct CudaEngine {
 
     // returns false on abort
     __device__ bool block(const KernelArgs &a, const Shared &sh, int s, uint32_t par, int nv, float *pbuf,
-                          const SlotRef &sr, uint32_t u_off, int lane)
+                          const SlotRef &sr, uint32_t u_off, int lane, uint32_t &gcache)
     {
         const uint8_t *kt = sh.kv + (size_t)s * sh.L.stage_bytes;
         const uint8_t *vt = kt + sh.L.tile_bytes;
@@ -564,7 +619,7 @@ struct CudaEngine {
             l += __shfl_xor_sync(0xffffffffu, l, off);
         __syncwarp();
 
-        if (!warp_wait<false>(sh.full_v(s, a.S), par, sh.abort, a.timeout_ns, a.device_status))
+        if (!warp_wait<false>(sh.full_v(s), par, sh.abort, a.timeout_ns, a.device_status))
             return false;
         float acc[GMAX][DE];
 #pragma unroll
@@ -588,9 +643,14 @@ struct CudaEngine {
         }
         __syncwarp();
         if (lane == 0)
-            mbar_arrive(sh.empty(s, a.S));
+            mbar_arrive(sh.empty(s));
 
         // block state into the leader's slot, counted on its ready barrier
+        if (sr.need) {
+            const int g = slot_gate(a, sh, sr, gcache);
+            if (g <= 0)
+                return g == 0;
+        }
         if (lane == 0) {
             mbar_arrive_expect_tx_cluster(sr.ready, slot_tx_bytes(a.G, D, GMAX, kEngineCuda));
             st_async_b32(sr.base, 0u, sr.ready);
@@ -661,7 +721,7 @@ struct MmaEngine {
     }
 
     __device__ bool block(const KernelArgs &a, const Shared &sh, int s, uint32_t par, int nv, float *,
-                          const SlotRef &sr, uint32_t u_off, int lane)
+                          const SlotRef &sr, uint32_t u_off, int lane, uint32_t &gcache)
     {
         const int r = lane >> 2, c = lane & 3;
         uint8_t *kt = sh.kv + (size_t)s * sh.L.stage_bytes;
@@ -753,7 +813,7 @@ struct MmaEngine {
                 }
             }
 
-        if (!warp_wait<false>(sh.full_v(s, a.S), par, sh.abort, a.timeout_ns, a.device_status))
+        if (!warp_wait<false>(sh.full_v(s), par, sh.abort, a.timeout_ns, a.device_status))
             return false;
         if (nv < PAGE) {
             // rows past the sequence end may hold anything: zero them so 0 * x = 0
@@ -787,7 +847,7 @@ struct MmaEngine {
             }
         __syncwarp();
         if (lane == 0)
-            mbar_arrive(sh.empty(s, a.S));
+            mbar_arrive(sh.empty(s));
 
         // columns of this lane after combining hi and lo: heads gA, gA+1
         const int gA = kShared ? 2 * (c & 1) : 2 * c;
@@ -804,6 +864,11 @@ struct MmaEngine {
             }
         // slot layout of this engine: 16-byte vectors, vector (dt, r, c) holds
         // u[gA][d], u[gA+1][d], u[gA][d+8], u[gA+1][d+8] with d = 16 dt + r
+        if (sr.need) {
+            const int g = slot_gate(a, sh, sr, gcache);
+            if (g <= 0)
+                return g == 0;
+        }
         if (lane == 0) {
             mbar_arrive_expect_tx_cluster(sr.ready, slot_tx_bytes(a.G, D, GMAX, kEngineMma));
             st_async_b32(sr.base, 0u, sr.ready);
@@ -837,15 +902,19 @@ template <typename T, int D, int PAGE, int GMAX, int ENGINE>
 using EngineFor = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX>,
                                             CudaEngine<T, D, PAGE, GMAX>>::type;
 
-// eng holds the unit's queries, loaded before the set-up barriers
-template <typename T, int D, int PAGE, int GMAX, int ENGINE>
+// eng holds the unit's queries, loaded before the set-up barriers.  GATE:
+// the window reaches past the state ring, so a finished state waits for its
+// slot (slot_gate).
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, bool GATE = false>
 __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h, int cw,
                              EngineFor<T, D, PAGE, GMAX, ENGINE> &eng)
 {
     const int lane = threadIdx.x & 31;
     float *pbuf = sh.pbuf + (ENGINE == kEngineMma ? 0 : cw * PAGE * GMAX);
-    const uint32_t ring_cl = mapa(smem_u32(sh.ring), 0);
-    const uint32_t ready_cl = mapa(sh.ready(0, a.S), 0);
+    const uint32_t ring_cl = mapa(sh.ring_leader, 0);
+    const uint32_t ready_cl = mapa(sh.ready_leader, 0);
+    const uint32_t ctrl_cl = mapa(smem_u32((const void *)sh.ctrl), 0);
+    uint32_t gcache = 0;
     for (uint32_t i = (uint32_t)cw;; i += (uint32_t)a.NW) {
         const int s = (int)(i % (uint32_t)a.S);
         const uint32_t par = (i / (uint32_t)a.S) & 1u;
@@ -856,18 +925,26 @@ __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h
             break;
         const int nv = (int)sh.stage_nv[s];
         const uint32_t slot = j % (uint32_t)a.R;
-        SlotRef sr{ring_cl + slot * sh.L.slot_bytes, ready_cl + 8u * slot};
+        const uint32_t need = (GATE && j >= (uint32_t)a.R) ? j - (uint32_t)a.R + 1u : 0u;
+        SlotRef sr{ring_cl + slot * sh.L.slot_bytes, ready_cl + 8u * slot, need, ctrl_cl};
         if (nv < 0) {  // bad page: forward the flag, free the stage
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(sh.empty(s, a.S));
+                mbar_arrive(sh.empty(s));
+            if (sr.need) {
+                const int g = slot_gate(a, sh, sr, gcache);
+                if (g < 0)
+                    break;
+                if (g == 0)
+                    continue;
+            }
             if (lane == 0) {
                 mbar_arrive_expect_tx_cluster(sr.ready, 4u);
                 st_async_b32(sr.base, 1u, sr.ready);
             }
             continue;
         }
-        if (!eng.block(a, sh, s, par, nv, pbuf, sr, sh.L.u_off_floats, lane))
+        if (!eng.block(a, sh, s, par, nv, pbuf, sr, sh.L.u_off_floats, lane, gcache))
             break;
     }
 }
@@ -952,7 +1029,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 {
     using MS = MergeShape<D, GMAX, ENGINE, NMW>;
     using Lay = typename MS::Lay;
-    constexpr int NVW = MS::NVW, VW = Lay::VW, VP = VW / 2, KB = MS::KB, NM = MS::NM, KH = MS::KH, NH = MS::NH;
+    constexpr int NVW = MS::NVW, VW = Lay::VW, KB = MS::KB, NM = MS::NM, KH = MS::KH, NH = MS::NH;
     static_assert(KB <= 8, "two partial sums per block in 16 lanes");
     const int lane = threadIdx.x & 31;
     const int G = a.G;
@@ -969,54 +1046,63 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
     // the running softmax scalars of head gl
     const int kl = lane / GMAX, gl = lane % GMAX;
     float Mx = -CUDART_INF_F, Lm = 0.f;
-    // running output of this lane's elements, as packed fp32 pairs
-    uint64_t o[NVW][VP];
+    // running output of this lane's elements (element e of vector i).  Scalar
+    // fp32: in these short dependent chains it runs faster than the packed
+    // f32x2 forms, and rounds identically.
+    float o[NVW][VW];
 #pragma unroll
     for (int i = 0; i < NVW; ++i)
 #pragma unroll
-        for (int q = 0; q < VP; ++q)
-            o[i][q] = 0ull;
+        for (int e = 0; e < VW; ++e)
+            o[i][e] = 0.f;
 
     int cnt = 0, stop = 0;
     bool failed = false;
     if (a.debug_flags & 1) {
         // a wait nothing will ever satisfy: exercises the bounded-wait path
-        if (!warp_wait<true>(sh.never(a.S, a.R), 0u, sh.abort, a.timeout_ns, a.device_status))
+        if (!warp_wait<true>(sh.never(), 0u, sh.abort, a.timeout_ns, a.device_status))
             failed = true;
     }
 
-    auto load_u = [&](const float *sp, uint64_t (&uv)[NVW][VP]) {
+    auto load_u = [&](const float *sp, float (&uv)[NVW][VW]) {
 #pragma unroll
         for (int ii = 0; ii < NVW; ++ii) {
             const float *up = sp + u_off + Lay::off(lane, vbase + ii);
             if constexpr (VW == 4) {
                 const float4 x = *reinterpret_cast<const float4 *>(up);
-                uv[ii][0] = pk2(x.x, x.y);
-                uv[ii][1] = pk2(x.z, x.w);
+                uv[ii][0] = x.x;
+                uv[ii][1] = x.y;
+                uv[ii][2] = x.z;
+                uv[ii][3] = x.w;
             } else {
                 const float2 x = *reinterpret_cast<const float2 *>(up);
-                uv[ii][0] = pk2(x.x, x.y);
+                uv[ii][0] = x.x;
+                uv[ii][1] = x.y;
             }
         }
     };
     // Fold batch block k into this warp's slice: Delta = beta (u - o),
-    // o += Delta; with sums, add o.Delta and |Delta|^2 of the slice to pd, pe.
-    auto fold = [&](int k, float beta, uint64_t bq, const uint64_t (&uv)[NVW][VP], float &pd, float &pe,
+    // o += Delta; with sums, add o.Delta and |Delta|^2 of the slice to pd, pe
+    // (accumulated over the even and the odd elements apart, then added).
+    // b0, b1: the shares of the lane's two heads (two-head layouts).
+    auto fold = [&](int k, float beta, float b0, float b1, const float (&uv)[NVW][VW], float &pd, float &pe,
                     bool sums) {
-        uint64_t bp[NVW];
+        float bp[NVW][2];
         const int kr = NH > 1 ? k % KH : k;  // row of the scan lanes holding block k
-        if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads: bq = (beta, beta) of both
+        if constexpr (Lay::kTwoHeads) {  // elements alternate between two heads
 #pragma unroll
-            for (int ii = 0; ii < NVW; ++ii)
-                bp[ii] = bq;
+            for (int ii = 0; ii < NVW; ++ii) {
+                bp[ii][0] = b0;
+                bp[ii][1] = b1;
+            }
         } else {  // vector i holds head i
 #pragma unroll
             for (int ii = 0; ii < NVW; ++ii) {
                 const float bi = __shfl_sync(0xffffffffu, beta, kr * GMAX + vbase + ii);
-                bp[ii] = (vbase + ii < G) ? pk2(bi, bi) : 0ull;
+                bp[ii][0] = bp[ii][1] = (vbase + ii < G) ? bi : 0.f;
             }
         }
-        uint64_t sd = 0ull, se = 0ull;
+        float sd[2] = {0.f, 0.f}, se[2] = {0.f, 0.f};
 #pragma unroll
         for (int ii = 0; ii < NVW; ++ii) {
             // the CUDA-core engine writes no state for padding rows (vector
@@ -1025,39 +1111,41 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
             if (!Lay::kTwoHeads && vbase + ii >= G)
                 continue;
 #pragma unroll
-            for (int q = 0; q < VP; ++q) {
-                // o += beta (u - o) as one fused step (one rounding); written
-                // as such so that no instantiation fuses it differently
-                const uint64_t df = sub2(uv[ii][q], o[ii][q]);
+            for (int e = 0; e < VW; ++e) {
+                // o += beta (u - o) as one fused step (one rounding), written
+                // with explicit roundings so that every instantiation computes
+                // exactly this
+                const float bb = bp[ii][e & 1];
+                const float df = __fsub_rn(uv[ii][e], o[ii][e]);
                 if (sums) {
-                    const uint64_t dl = mul2(bp[ii], df);
-                    sd = fma2(o[ii][q], dl, sd);
-                    se = fma2(dl, dl, se);
+                    const float dl = __fmul_rn(bb, df);
+                    sd[e & 1] = __fmaf_rn(o[ii][e], dl, sd[e & 1]);
+                    se[e & 1] = __fmaf_rn(dl, dl, se[e & 1]);
                 }
-                o[ii][q] = fma2(bp[ii], df, o[ii][q]);
+                o[ii][e] = __fmaf_rn(bb, df, o[ii][e]);
             }
         }
         if (sums) {
-            pd = lo2(sd) + hi2(sd);
-            pe = lo2(se) + hi2(se);
+            pd = __fadd_rn(sd[0], sd[1]);
+            pe = __fadd_rn(se[0], se[1]);
         }
     };
     // fold blocks 0..kend of the batch starting at slot s0 (u loads one block ahead)
     auto fold_batch = [&](int s0, int kend, float beta, float beta_hi, float (&v)[16], bool sums) {
-        uint64_t ua[NVW][VP], ub[NVW][VP];
+        float ua[NVW][VW], ub[NVW][VW];
         load_u(sh.ring + (size_t)s0 * slot_floats, ua);
-        // the beta pairs of every block of the batch, fetched before the fold
-        // so that the shuffles stay off the chain that carries o from block to block
-        uint64_t bq[KB];
+        // the shares of every block of the batch, fetched before the fold so
+        // that the shuffles stay off the chain that carries o from block to block
+        float bq0[KB], bq1[KB];
 #pragma unroll
         for (int k = 0; k < KB; ++k) {
-            bq[k] = 0ull;
+            bq0[k] = bq1[k] = 0.f;
             if constexpr (Lay::kTwoHeads) {
                 const float bk = (NH > 1 && k >= KH) ? beta_hi : beta;
                 const int kr = NH > 1 ? k % KH : k;
                 const int h0 = Lay::head(lane, 0, 0);
-                bq[k] = pk2(__shfl_sync(0xffffffffu, bk, kr * GMAX + h0),
-                            __shfl_sync(0xffffffffu, bk, kr * GMAX + h0 + 1));
+                bq0[k] = __shfl_sync(0xffffffffu, bk, kr * GMAX + h0);
+                bq1[k] = __shfl_sync(0xffffffffu, bk, kr * GMAX + h0 + 1);
             }
         }
 #pragma unroll
@@ -1069,7 +1157,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
                 sn = sn >= a.R ? sn - a.R : sn;
                 load_u(sh.ring + (size_t)sn * slot_floats, (k & 1) ? ua : ub);
             }
-            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, bq[k], (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1], sums);
+            fold(k, (NH > 1 && k >= KH) ? beta_hi : beta, bq0[k], bq1[k], (k & 1) ? ub : ua, v[2 * k], v[2 * k + 1],
+                 sums);
         }
     };
 
@@ -1095,7 +1184,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         if (mw == 0) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk, a.S), pk);
+                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk), pk);
                 if (__any_sync(0xffffffffu, arrived && __float_as_uint(spk[0]) != 0u)) {
                     local_fail = true;
                     break;
@@ -1141,7 +1230,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         for (int q = 0; q < 16; ++q)
             v[q] = 0.f;
         float beta = 0.f, beta_hi = 0.f, n0part = 0.f;  // beta_hi: blocks KH.. (two scan rows)
-        uint64_t o0[NVW][VP];
+        float o0[NVW][VW];
         if (!local_fail) {
             // 2. shares of the softmax mass: beta_(k,g) = w_k / (L_prev + w_0 + ... + w_k)
             float Mb;
@@ -1222,15 +1311,15 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
             Mx = Mb;
             if constexpr (DET) {
                 // 3. ||o||^2 before the batch, then fold the batch into this warp's slice
-                uint64_t n2 = 0ull;
+                float n2[2] = {0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < NVW; ++i)
 #pragma unroll
-                    for (int q = 0; q < VP; ++q) {
-                        o0[i][q] = o[i][q];
-                        n2 = fma2(o[i][q], o[i][q], n2);
+                    for (int e = 0; e < VW; ++e) {
+                        o0[i][e] = o[i][e];
+                        n2[e & 1] = __fmaf_rn(o[i][e], o[i][e], n2[e & 1]);
                     }
-                n0part = lo2(n2) + hi2(n2);
+                n0part = __fadd_rn(n2[0], n2[1]);
             }
             fold_batch(s0, nb - 1, beta, beta_hi, v, DET);
         }
@@ -1307,8 +1396,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
             const float d_scale = __fdividef(fabsf(t), (r1 + r0) * r0);
             const float pr = Dp * i0;  // component of Delta along o_{j-1}
             const float x = r0 + pr;
-            const float y2 = fmaxf(Ep - pr * pr, 0.f);
-            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : 1.f - x * i1;
+            const float y2 = fmaxf(fmaf(-pr, pr, Ep), 0.f);
+            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : fmaf(-x, i1, 1.f);
             stable = (d_scale < eps_m) && (d_dir < eps_d);
         }
         // 6. patience over the batch, one lane per block: the counter after
@@ -1329,8 +1418,8 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
 #pragma unroll
                 for (int i = 0; i < NVW; ++i)
 #pragma unroll
-                    for (int q = 0; q < VP; ++q)
-                        o[i][q] = o0[i][q];
+                    for (int e = 0; e < VW; ++e)
+                        o[i][e] = o0[i][e];
                 fold_batch(s0, kstop, beta, beta_hi, v, false);
             }
         }
@@ -1357,7 +1446,7 @@ __device__ void merge_role(const KernelArgs &a, const Shared &sh, int b, int h, 
         for (int e = 0; e < VW; ++e) {
             const int i = vbase + ii;
             const int g = Lay::head(lane, i, e);
-            const float val = (e & 1) ? hi2(o[ii][e >> 1]) : lo2(o[ii][e >> 1]);
+            const float val = o[ii][e];
             if (g < G && (Lay::kTwoHeads || i < G))
                 op[(int64_t)(h * G + g) * a.out_sh + Lay::dim(lane, i, e)] = failed ? 0.f : val;
         }
@@ -1431,7 +1520,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
     uint32_t done = 0u;  // bit t: token t has stopped (the same in every lane)
     bool failed = false;
     if (a.debug_flags & 1) {
-        if (!warp_wait<true>(sh.never(a.S, a.R), 0u, sh.abort, a.timeout_ns, a.device_status))
+        if (!warp_wait<true>(sh.never(), 0u, sh.abort, a.timeout_ns, a.device_status))
             failed = true;
     }
 
@@ -1552,7 +1641,7 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
         if (mw == 0) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk, a.S), pk);
+                const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk), pk);
                 if (__any_sync(0xffffffffu, arrived && __float_as_uint(spk[0]) != 0u)) {
                     local_fail = true;
                     break;
@@ -1738,8 +1827,8 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
             const float d_scale = __fdividef(fabsf(tt), (r1 + r0) * r0);
             const float pr = Dp * i0;
             const float x = r0 + pr;
-            const float y2 = fmaxf(Ep - pr * pr, 0.f);
-            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : 1.f - x * i1;
+            const float y2 = fmaxf(fmaf(-pr, pr, Ep), 0.f);
+            const float d_dir = x > 0.f ? __fdividef(y2, r1 * (r1 + x)) : fmaf(-x, i1, 1.f);
             stable = (d_scale < eps_m) && (d_dir < eps_d);
         }
         // 6. patience per token, one lane per block (as in merge_role)
@@ -1851,7 +1940,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     sh.red = reinterpret_cast<float *>(base + sh.L.red_off);
     sh.stage_j = reinterpret_cast<uint32_t *>(base + sh.L.meta_off);
     sh.stage_nv = sh.stage_j + a.S;
-    sh.bar0 = smem_u32(base + sh.L.bar_off);
+    const uint32_t bar0 = smem_u32(base + sh.L.bar_off);
+    sh.bar_full_k = bar0;
+    sh.bar_full_v = bar0 + 8u * a.S;
+    sh.bar_empty = bar0 + 16u * a.S;
+    sh.bar_ready = bar0 + 24u * a.S;
+    sh.bar_never = bar0 + 8u * (3 * a.S + a.R);
+    sh.ring_leader = smem_u32(sh.ring);
+    sh.ready_leader = sh.bar_ready;
     sh.ctrl = reinterpret_cast<volatile uint32_t *>(base + sh.L.ctrl_off);
     sh.fetched = sh.ctrl + 1;
     sh.abort = sh.ctrl + 2;
@@ -1889,12 +1985,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.S; ++s) {
             mbar_init(sh.full_k(s), 1);
-            mbar_init(sh.full_v(s, a.S), 1);
-            mbar_init(sh.empty(s, a.S), 1);
+            mbar_init(sh.full_v(s), 1);
+            mbar_init(sh.empty(s), 1);
         }
         for (int r = 0; r < a.R; ++r)
-            mbar_init(sh.ready(r, a.S), 1);
-        mbar_init(sh.never(a.S, a.R), 1);
+            mbar_init(sh.ready(r), 1);
+        mbar_init(sh.never(), 1);
         sh.ctrl[0] = 0u;
         sh.ctrl[1] = 0u;
         sh.ctrl[2] = 0u;
@@ -1907,7 +2003,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
     if (walk) {
         if (warp == 0)
-            producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank, first_lb, first_pp);
+            producer_role<T, D, PAGE, ENGINE>(a, sh, &tmk, &tmv, b, h, N, Lseq, rank, a.C, first_lb, first_pp);
         else if (warp <= NM) {
             if (rank == 0) {
                 if constexpr (NQ == 1)

@@ -21,6 +21,8 @@ KernelFn f32_cuda(int gmax, int d, int page, bool detector);
 KernelFn bf16_cuda(int gmax, int d, int page);
 // bf16 caches, tensor-core block engine (gmax 4 or 8; nmw 1 or 4 merge warps)
 KernelFn bf16_mma(int gmax, int nmw, int d, int page, bool detector);
+// bf16 caches, tensor-core block engine, dedicated merge CTA (gmax 4 or 8)
+KernelFn bf16_mma_dl(int gmax, int d, int page, bool detector);
 // two query tokens sharing one walk (head dim 128)
 KernelFn multi(bool f32, int engine, int page, int gmax, int nmw);
 

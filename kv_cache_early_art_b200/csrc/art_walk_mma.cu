@@ -1,6 +1,7 @@
 // art_walk_mma.cu -- walk kernel instantiations for bf16 caches on the
 // tensor-core block engine.
 #include "art_walk.h"
+#include "art_walk_dl.cuh"
 
 namespace art_walk {
 
@@ -34,6 +35,18 @@ KernelFn bf16_mma(int gmax, int nmw, int d, int page, bool detector)
     if (nmw == 4)
         return gmax == 4 ? by_dp<4, 4>(d, page) : by_dp<8, 4>(d, page);
     return gmax == 4 ? by_dp<4, 1>(d, page) : by_dp<8, 1>(d, page);
+}
+
+KernelFn bf16_mma_dl(int gmax, int d, int page, bool detector)
+{
+    using art::art_walk_dl_kernel;
+    using T = __nv_bfloat16;
+    constexpr int E = art::kEngineMma;
+    if (d != 128 || page != 64)
+        return nullptr;
+    if (detector)
+        return gmax == 4 ? art_walk_dl_kernel<T, 128, 64, 4, E, 4, true> : art_walk_dl_kernel<T, 128, 64, 8, E, 8, true>;
+    return gmax == 4 ? art_walk_dl_kernel<T, 128, 64, 4, E, 4, false> : art_walk_dl_kernel<T, 128, 64, 8, E, 8, false>;
 }
 
 }  // namespace art_walk
