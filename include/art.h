@@ -117,7 +117,8 @@ typedef struct {
                            /* pages read past the stop)                                    */
     int32_t smem_bytes;    /* dynamic shared memory per CTA                               */
     int32_t prefetch;      /* further blocks pulled into L2 ahead of the staged ones      */
-    int32_t merge_cta;     /* 1: the cluster's first CTA only merges                      */
+    int32_t merge_cta;     /* 1: the cluster's first CTA only merges; 2: one merge CTA    */
+                           /* per unit reached through the workspace                      */
     int32_t ring_slots;    /* block states the merging CTA holds (= window, or fewer with */
                            /* merge_cta: then a finished state waits for a free slot)     */
 } art_launch_info_t;
@@ -172,6 +173,19 @@ typedef struct {
                                    /* 1 elsewhere returns ART_ERR_UNSUPPORTED, and with     */
                                    /* cluster_size 1 ART_ERR_PARAM.  Stops and outputs are  */
                                    /* the sequential rule's, as with every launch shape.    */
+                                   /* 2: the same merge, reached through the workspace      */
+                                   /* below instead of a cluster, so that more CTAs serve   */
+                                   /* each unit (one merge CTA and W fetching CTAs per      */
+                                   /* unit, all resident at once: a cooperative launch).    */
+                                   /* Only on request; 2 without a workspace returns        */
+                                   /* ART_ERR_NULL, with one too small ART_ERR_SHAPE.       */
+    void *workspace;               /* device memory or NULL: scratch for merge_cta = 2      */
+                                   /* (block states, ready tags and counters; at least      */
+                                   /* art_workspace_bytes(p) bytes, 256-byte aligned).  It  */
+                                   /* needs no clearing: every word is tagged with the      */
+                                   /* call.  Calls that overlap on the GPU must not share   */
+                                   /* one workspace.                                        */
+    int64_t workspace_bytes;       /* its size                                              */
 } art_params_t;
 
 /*
@@ -180,6 +194,16 @@ typedef struct {
  * overrides.  Passing zeros for every option reproduces art_decode_attention.
  */
 art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream);
+
+/*
+ * art_workspace_bytes -- the workspace art_decode_attention_ex can use for
+ * this problem with merge_cta = 2: the tensors, options and
+ * current device of p decide it.  Returns 0 when that walk does not apply
+ * (more units than SMs, a cache type, head dim or page size it is not built
+ * for, several query tokens), a negative art_status_t when the arguments are
+ * invalid.  Nothing is launched.
+ */
+int64_t art_workspace_bytes(const art_params_t *p);
 
 /*
  * art_decode_attention_multi -- n_queries query tokens of each sequence (for

@@ -58,7 +58,8 @@ class ArtParams(ctypes.Structure):
         ("engine", ctypes.c_int32), ("cluster_size", ctypes.c_int32), ("stages", ctypes.c_int32),
         ("compute_warps", ctypes.c_int32), ("window", ctypes.c_int32), ("timeout_ns", ctypes.c_int64),
         ("debug_flags", ctypes.c_int32), ("info", ctypes.POINTER(ArtLaunchInfo)), ("prefetch", ctypes.c_int32),
-        ("detector_off", ctypes.c_int32), ("merge_cta", ctypes.c_int32)]
+        ("detector_off", ctypes.c_int32), ("merge_cta", ctypes.c_int32), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_int64)]
 
 
 _P = ctypes.POINTER
@@ -77,6 +78,8 @@ _lib.art_page_summary.restype = ctypes.c_int
 _lib.art_build_order_importance.argtypes = [_P(ArtTensor)] * 4 + [ctypes.c_int32, ctypes.c_float] + [
     _P(ArtTensor)] * 2 + [ctypes.c_void_p, ctypes.c_void_p]
 _lib.art_build_order_importance.restype = ctypes.c_int
+_lib.art_workspace_bytes.argtypes = [_P(ArtParams)]
+_lib.art_workspace_bytes.restype = ctypes.c_int64
 _lib.art_strerror.argtypes = [ctypes.c_int]
 _lib.art_strerror.restype = ctypes.c_char_p
 _lib.art_version.argtypes = []
@@ -184,10 +187,11 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
                             P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
                             P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
                             engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
-                            debug_flags=0, prefetch=0, detector_off=0, merge_cta=0, out=None, stop_block=None,
-                            stream=None, want_info=False):
+                            debug_flags=0, prefetch=0, detector_off=0, merge_cta=0, workspace=None, out=None,
+                            stop_block=None, stream=None, want_info=False):
     """art_decode_attention_ex in art.h.  Per-sequence arrays are device
-    tensors of length B (float32 thresholds, int32 P / min_blocks).
+    tensors of length B (float32 thresholds, int32 P / min_blocks);
+    workspace a device tensor (any dtype, 256-byte aligned) or None.
     Returns (out, stop_block) or (out, stop_block, launch_info_dict)."""
     B, Hq, d = q.shape
     if out is None:
@@ -198,6 +202,10 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
                       timeout_ns, debug_flags, prefetch, detector_off, merge_cta)
+    if workspace is not None:
+        _need_cuda(workspace)
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
     st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
     _check(st, "art_decode_attention_ex")
     if want_info:
@@ -228,6 +236,28 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
     if want_info:
         return out, stop_block, info.as_dict()
     return out, stop_block
+
+
+def art_workspace_bytes(q, k_cache, v_cache, page_table, block_order, seq_lens, **options):
+    """art_workspace_bytes in art.h: the workspace art_decode_attention_ex can
+    use for this problem (0 when its workspace walk does not apply)."""
+    B, Hq, d = q.shape
+    out = options.pop("out", None)
+    stop_block = options.pop("stop_block", None)
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    kw = dict(eps_m=0.0, eps_d=0.0, P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
+              P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None, engine=0,
+              cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0, debug_flags=0, prefetch=0,
+              detector_off=0, merge_cta=0)
+    kw.update(options)
+    p, _ = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, **kw)
+    n = int(_lib.art_workspace_bytes(ctypes.byref(p)))
+    if n < 0:
+        raise ArtError(n, "art_workspace_bytes")
+    return n
 
 
 def art_build_order_sink_recency(seq_lens, page, block_order=None, max_blocks=None, stream=None):

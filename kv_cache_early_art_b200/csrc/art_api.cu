@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <type_traits>
@@ -14,6 +15,7 @@
 #include "art_kernels.cuh"
 #include "art_walk.h"
 #include "art_walk_dl.cuh"
+#include "art_walk_gr.cuh"
 
 namespace {
 
@@ -172,10 +174,13 @@ art_status_t check_params(const art_params_t *p)
     if (p->engine < 0 || p->engine > 2 || p->cluster_size < 0 || p->cluster_size > 16 || p->stages < 0 ||
         p->stages > 8 || p->compute_warps < 0 || p->compute_warps > art::kMaxComputeWarps || p->window < 0 ||
         p->window > 128 || p->timeout_ns < 0 || (p->debug_flags & ~1) || p->prefetch < -1 || p->prefetch > 64 ||
-        p->detector_off < 0 || p->detector_off > 1 || p->merge_cta < -1 || p->merge_cta > 1)
+        p->detector_off < 0 || p->detector_off > 1 || p->merge_cta < -1 || p->merge_cta > 2 ||
+        p->workspace_bytes < 0)
         return ART_ERR_PARAM;
     if (p->stages == 1 || (p->window > 0 && p->window < art::kMinWindow))
         return ART_ERR_PARAM;
+    if (p->workspace && !aligned(p->workspace, 256))
+        return ART_ERR_SHAPE;
     for (const void *ptr : {(const void *)p->eps_m_per_seq, (const void *)p->eps_d_per_seq,
                             (const void *)p->P_per_seq, (const void *)p->min_blocks_per_seq,
                             (const void *)p->blocks_fetched, (const void *)p->device_status})
@@ -320,7 +325,8 @@ art_status_t make_cache_map(CUtensorMap *map, const art_tensor_t *c, int dtype, 
 struct Shape {
     int engine, gmax, nmw, S, NW, R, C, PF, smem, threads;
     int RF = 0;              // window (blocks fetched ahead of the merged prefix); R = ring slots
-    int dl = 0;              // 1: dedicated merge CTA (art_walk_dl_kernel)
+    int dl = 0;              // 1: dedicated merge CTA (art_walk_dl_kernel); 2: through the workspace
+    int W = 0, Rg = 0;       // workspace walk: fetching CTAs per unit, ring slots per unit
     KernelFn fn = nullptr;   // set by the dedicated-merge choice
 };
 
@@ -570,6 +576,104 @@ art_status_t choose_dl(const art_params_t *p, const Problem &pr, const DeviceInf
     return ART_OK;
 }
 
+// The dedicated merge reached through a workspace (art_walk_gr_kernel), on
+// request (merge_cta = 2): one merge CTA and W fetching CTAs per unit, as many
+// as fit on the GPU at once (the launch is cooperative).  need: the workspace
+// this problem can use (a ring of 128 slots per unit), also when none is
+// given.  *chosen stays false when another walk should run instead.
+art_status_t choose_gr(const art_params_t *p, const Problem &pr, const DeviceInfo &di, Shape *out, bool *chosen,
+                       int64_t *need)
+{
+    *chosen = false;
+    *need = 0;
+    const bool forced = p->merge_cta == 2;
+    const int engine = p->engine ? p->engine : (pr.dtype == ART_BF16 ? art::kEngineMma : art::kEngineCuda);
+    if (engine != art::kEngineMma || pr.dtype != ART_BF16 || pr.d != 128 || pr.page != 64)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    const int units = pr.B * pr.Hkv;
+    if (!forced && units >= di.sms)
+        return ART_OK;
+    if (p->compute_warps && p->stages && p->stages % p->compute_warps != 0)
+        return ART_ERR_PARAM;
+    Shape s;
+    s.engine = art::kEngineMma;
+    s.gmax = gmax_for(pr.G, s.engine);
+    s.nmw = s.gmax;
+    s.PF = p->prefetch > 0 ? p->prefetch : 0;
+    s.dl = 2;
+    const int es = (int)elem_size(pr.dtype);
+    const int limit = di.smem_optin - 1024;
+    // the merge CTA's staging ring: at least five merge batches deep (a batch
+    // is copied in only once the batch five before it has been decided)
+    int R = 64;
+    for (; R > 40; R -= 8)
+        if ((int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total <= limit)
+            break;
+    if ((int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total > limit)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    s.R = R;
+    static const int cand[][2] = {{6, 6}, {3, 6}, {5, 5}, {4, 4}, {2, 4}, {2, 2}, {1, 2}};
+    bool fit = false;
+    for (const auto &c : cand) {
+        int NW = p->compute_warps ? p->compute_warps : c[0];
+        int S = p->stages ? p->stages : c[1];
+        if (p->stages && !p->compute_warps) {
+            while (S % NW != 0)
+                --NW;
+        } else if (!p->stages) {
+            S = NW * ((S + NW - 1) / NW);
+            if (S > 8)
+                S = NW * (8 / NW);
+        }
+        if ((int)art::make_dl_layout(S, R, pr.page, pr.d, es, s.gmax, 0).total <= limit) {
+            s.NW = NW;
+            s.S = S;
+            fit = true;
+            break;
+        }
+    }
+    if (!fit)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    const int lead = (int)art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).total;
+    const int work = (int)art::make_dl_layout(s.S, R, pr.page, pr.d, es, s.gmax, 0).total;
+    s.smem = (lead > work ? lead : work) + 1024;
+    s.threads = 32 * (2 + s.nmw > 1 + s.NW ? 2 + s.nmw : 1 + s.NW);
+    s.fn = art_walk::bf16_mma_gr(s.gmax, pr.d, pr.page, !p->detector_off);
+    if (!s.fn)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    art_status_t st = prepare_kernel(s.fn, s.smem);
+    if (st != ART_OK)
+        return st;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, s.fn, s.threads, s.smem) != cudaSuccess) {
+        cudaGetLastError();
+        return ART_ERR_LAUNCH;
+    }
+    const int slots = di.sms * (per_sm < 1 ? 0 : per_sm);
+    const int W = p->cluster_size ? p->cluster_size - 1 : (slots / units) - 1;
+    if (W < (forced ? 1 : 3) || (int64_t)units * (1 + W) > slots)
+        return forced ? ART_ERR_UNSUPPORTED : ART_OK;
+    s.W = W;
+    s.C = 1 + W;
+    const uint32_t slot = art::make_dl_layout(0, R, pr.page, pr.d, es, s.gmax, R).slot_bytes;
+    *need = art::gr_workspace_bytes(units, W, 128, slot);
+    if (!p->workspace)
+        return forced ? ART_ERR_NULL : ART_OK;
+    int Rg = 128;
+    while (Rg > 16 && art::gr_workspace_bytes(units, W, Rg, slot) > p->workspace_bytes)
+        Rg -= 8;
+    if (art::gr_workspace_bytes(units, W, Rg, slot) > p->workspace_bytes)
+        return forced ? ART_ERR_SHAPE : ART_OK;
+    s.Rg = Rg;
+    // the window: blocks fetched ahead of the merged count, within the ring
+    s.RF = p->window ? (p->window < Rg ? p->window : Rg) : Rg;
+    *out = s;
+    *chosen = true;
+    return ART_OK;
+}
+
+std::atomic<uint32_t> g_epoch{0};
+
 // tokens_dim: q and out are [B, T, Hq, d] and stop_block [B, T, Hkv] (T = nq)
 art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool tokens_dim = false)
 {
@@ -590,12 +694,19 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
         return ART_ERR_UNSUPPORTED;
     if (nq > 1 && p->merge_cta == 1)
         return ART_ERR_UNSUPPORTED;
+    if (nq > 1 && p->merge_cta == 2)
+        return ART_ERR_UNSUPPORTED;
     Shape s;
-    bool dl = false;
-    if (nq == 1 && p->merge_cta != -1 && (st = choose_dl(p, pr, di, &s, &dl)) != ART_OK)
+    bool dl = false, gr = false;
+    if (nq == 1 && p->merge_cta == 2) {
+        int64_t need = 0;
+        if ((st = choose_gr(p, pr, di, &s, &gr, &need)) != ART_OK)
+            return st;
+    }
+    if (!gr && nq == 1 && p->merge_cta != -1 && p->merge_cta != 2 && (st = choose_dl(p, pr, di, &s, &dl)) != ART_OK)
         return st;
     KernelFn fn = nullptr;
-    if (dl) {
+    if (dl || gr) {
         fn = s.fn;
     } else {
         if ((st = choose_shape(p, pr, di, &s)) != ART_OK)
@@ -652,13 +763,29 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     ka.out_st = pr.out_st;
     ka.stop_st = pr.stop_st;
 
-    if (!dl && (st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
+    if (!dl && !gr && (st = pick_cluster(fn, &s, pr, di, ka)) != ART_OK)
         return st;
     ka.C = s.C;
     ka.S = s.S;
     ka.NW = s.NW;
     ka.R = s.R;
     ka.RF = s.RF;
+    if (gr) {
+        // the workspace: merged counts, fetch counts, ready tags, states
+        const int units = pr.B * pr.Hkv;
+        uint8_t *ws = static_cast<uint8_t *>(p->workspace);
+        ka.g_ctrl = reinterpret_cast<unsigned long long *>(ws);
+        ka.g_done = ka.g_ctrl + units;
+        ka.g_flags = ka.g_done + (int64_t)units * s.W;
+        const uintptr_t st0 = reinterpret_cast<uintptr_t>(ka.g_flags + (int64_t)units * s.Rg);
+        ka.g_states = reinterpret_cast<float *>((st0 + 255) & ~(uintptr_t)255);
+        uint32_t e = ++g_epoch;
+        if (e == 0)
+            e = ++g_epoch;  // 0 never tags a word (a fresh workspace may hold zeros)
+        ka.epoch = e;
+        ka.Rg = s.Rg;
+        ka.W = s.W;
+    }
     ka.PF = s.PF;
 
     CUtensorMap tmk, tmv;
@@ -681,6 +808,11 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (gr) {
+        // no clusters; every CTA resident at once (they wait on one another)
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
     if (p->info) {
         p->info->engine = s.engine;
         p->info->cluster_size = s.C;
@@ -689,7 +821,7 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
         p->info->stages = s.S;
         p->info->compute_warps = s.NW;
         p->info->window = s.RF;
-        p->info->ring_slots = s.R;
+        p->info->ring_slots = gr ? s.Rg : s.R;
         p->info->prefetch = s.PF;
         p->info->smem_bytes = s.smem;
         p->info->merge_cta = s.dl;
@@ -710,6 +842,31 @@ art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
     if (!p)
         return ART_ERR_NULL;
     return launch(p, stream);
+}
+
+int64_t art_workspace_bytes(const art_params_t *p)
+{
+    if (!p)
+        return ART_ERR_NULL;
+    Problem pr;
+    art_status_t st = check_tensors(p, &pr);
+    if (st != ART_OK)
+        return st;
+    if ((st = check_params(p)) != ART_OK)
+        return st;
+    DeviceInfo di;
+    if ((st = device_info(&di)) != ART_OK)
+        return st;
+    if (p->merge_cta == -1 || p->merge_cta == 1 || (p->merge_cta != 2 && pr.B * pr.Hkv >= di.sms))
+        return 0;
+    art_params_t q = *p;
+    q.merge_cta = 2;
+    q.workspace = nullptr;
+    Shape s;
+    bool chosen = false;
+    int64_t need = 0;
+    choose_gr(&q, pr, di, &s, &chosen, &need);
+    return need;
 }
 
 art_status_t art_decode_attention_multi(const art_params_t *p, int32_t n_queries, art_stream_t stream)

@@ -78,7 +78,22 @@ struct KernelArgs {
     // G = NQ * GQ rows per unit, row r is head r % GQ of token r / GQ
     int32_t NQ, GQ;
     int64_t q_st, out_st, stop_st;      // element strides between a sequence's tokens
+    // hand-over through a workspace in global memory (the walk whose merge
+    // CTA is not in the fetching CTAs' cluster): per unit the merged count,
+    // per fetching CTA its fetch count, per ring slot a ready tag and the
+    // block state.  Every word carries this call's epoch in its high half.
+    unsigned long long *g_ctrl, *g_done, *g_flags;
+    float *g_states;
+    uint32_t epoch;
+    int32_t Rg, W;                      // global ring slots per unit, fetching CTAs per unit
 };
+
+// merged count of a unit published in the workspace during this call (0 before)
+__device__ __forceinline__ uint32_t gm_merged(const KernelArgs &a, int unit)
+{
+    const unsigned long long v = ld_acquire_gpu_u64(a.g_ctrl + unit);
+    return (uint32_t)(v >> 32) == a.epoch ? (uint32_t)v : 0u;
+}
 
 // Shared-memory carve-up, identical on host and device.
 struct Layout {
@@ -270,10 +285,11 @@ struct Shared {
 // ---- producer ----------------------------------------------------------------
 
 // rank, C: this CTA's place among the CTAs that fetch for the unit and their
-// number (steps j = rank, rank + C, ... are this CTA's).  kAcquire: read the
-// merged progress with acquire semantics (needed where the warp that publishes
-// it is not the one that read the freed slots).
-template <typename T, int D, int PAGE, int ENGINE, bool kAcquire = false>
+// number (steps j = rank, rank + C, ... are this CTA's).  CTRL: where the
+// merged progress is read: 0 the cluster leader's shared memory (relaxed), 1
+// the same with acquire semantics (needed where the warp that publishes it is
+// not the one that read the freed slots), 2 the workspace in global memory.
+template <typename T, int D, int PAGE, int ENGINE, int CTRL = 0>
 __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUtensorMap *tmk, const CUtensorMap *tmv,
                               int b, int h, int N, int Lseq, uint32_t rank, int C, int first_lb, int first_pp)
 {
@@ -332,7 +348,9 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
         if (lane == 0 && ((uint32_t)j >= ctrl_cache + (uint32_t)R || (k & 3) == 0)) {
             uint64_t t0 = 0;
             for (uint32_t it = 0;; ++it) {
-                const uint32_t c = kAcquire ? ld_acquire_cluster_u32(ctrl_cl) : ld_relaxed_cluster_u32(ctrl_cl);
+                const uint32_t c = CTRL == 2   ? gm_merged(a, b * a.Hkv + h)
+                                   : CTRL == 1 ? ld_acquire_cluster_u32(ctrl_cl)
+                                               : ld_relaxed_cluster_u32(ctrl_cl);
                 if (c & kStopBit) { go = 0; break; }
                 ctrl_cache = c;
                 if ((uint32_t)j < c + (uint32_t)R) break;
@@ -458,8 +476,13 @@ __device__ void producer_role(const KernelArgs &a, const Shared &sh, const CUten
                 warp_wait<false>(sh.full_v(s), vphase >> s & 1u, sh.abort, a.timeout_ns, a.device_status, false);
         }
     }
-    if (lane == 0)
-        atom_add_cluster_u32(mapa(smem_u32((const void *)sh.fetched), 0), touched);
+    if (lane == 0) {
+        if constexpr (CTRL == 2)
+            st_release_gpu_u64(a.g_done + (int64_t)(b * a.Hkv + h) * a.W + rank,
+                               ((unsigned long long)a.epoch << 32) | touched);
+        else
+            atom_add_cluster_u32(mapa(smem_u32((const void *)sh.fetched), 0), touched);
+    }
 }
 
 // ---- block engines -------------------------------------------------------------
@@ -473,49 +496,108 @@ struct SlotRef {
     uint32_t ready;  // cluster address of its ready barrier
     uint32_t need;   // the slot is free once the merged count reaches this (0: it is free)
     uint32_t ctrl;   // cluster address of the merged count
+    // the same through the workspace: the slot, its ready tag and the tag
+    // written there once the state is complete, the unit's merged count
+    float *gslot;
+    unsigned long long *gflag;
+    unsigned long long tag;
+    int unit;
 };
 
 // Wait (whole warp, bounded) until the slot a finished block state goes to
 // is free: the block R places earlier in the walk has been merged.  Needed
-// only where the window reaches past the state ring.  Returns 1 to push, 0 to
-// drop the state (the walk has stopped, or failed, before it), -1 on timeout
-// or abort.  cache holds the last merged count this warp read.
-static __device__ __noinline__ int slot_gate(const KernelArgs &a, const Shared &sh, const SlotRef &sr, uint32_t &cache)
+// only where the window reaches past the state ring.  Takes and returns the
+// last merged count this warp read (kStopBit set once the walk has stopped
+// or failed: the state is then dropped), or kGateFailed on timeout or abort.
+constexpr uint32_t kGateFailed = 0x7fffffffu;
+
+static __device__ __noinline__ uint32_t slot_gate_wait(uint32_t need, uint32_t ctrl, uint32_t cache,
+                                                       volatile uint32_t *abort, int64_t timeout_ns,
+                                                       int32_t *status)
 {
-    int r = 0;
     if ((threadIdx.x & 31) == 0) {
         uint64_t t0 = 0;
         for (uint32_t it = 0;; ++it) {
-            if (cache & kStopBit) {
-                r = 0;
+            if ((cache & kStopBit) || cache >= need)
                 break;
-            }
-            if (cache >= sr.need) {
-                r = 1;
-                break;
-            }
-            cache = ld_acquire_cluster_u32(sr.ctrl);
+            cache = ld_acquire_cluster_u32(ctrl);
             if ((it & 15u) == 15u) {
                 const uint64_t now = global_timer_ns();
                 if (t0 == 0)
                     t0 = now;
-                if (*sh.abort) {
-                    r = -1;
+                if (*abort) {
+                    cache = kGateFailed;
                     break;
                 }
-                if ((int64_t)(now - t0) > a.timeout_ns) {
-                    *sh.abort = 1u;
-                    record_error(a.device_status, kErrTimeout);
-                    r = -1;
+                if ((int64_t)(now - t0) > timeout_ns) {
+                    *abort = 1u;
+                    record_error(status, kErrTimeout);
+                    cache = kGateFailed;
                     break;
                 }
             }
         }
     }
-    r = __shfl_sync(0xffffffffu, r, 0);
     cache = __shfl_sync(0xffffffffu, cache, 0);
     __syncwarp();  // the lanes' slot writes come after lane 0's acquire
-    return r;
+    return cache;
+}
+
+// 1: push the state; 0: drop it (the walk has stopped); -1: timeout or abort
+__device__ __forceinline__ int slot_gate(const KernelArgs &a, const Shared &sh, const SlotRef &sr, uint32_t &cache)
+{
+    cache = slot_gate_wait(sr.need, sr.ctrl, cache, sh.abort, a.timeout_ns, a.device_status);
+    return cache == kGateFailed ? -1 : ((cache & kStopBit) ? 0 : 1);
+}
+
+// The same wait on the merged count in the workspace.
+static __device__ __noinline__ uint32_t slot_gate_wait_gm(uint32_t need, const unsigned long long *ctrl,
+                                                          uint32_t epoch, uint32_t cache, volatile uint32_t *abort,
+                                                          int64_t timeout_ns, int32_t *status)
+{
+    if ((threadIdx.x & 31) == 0) {
+        uint64_t t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+            if ((cache & kStopBit) || cache >= need)
+                break;
+            const unsigned long long v = ld_acquire_gpu_u64(ctrl);
+            cache = (uint32_t)(v >> 32) == epoch ? (uint32_t)v : 0u;
+            if ((it & 15u) == 15u) {
+                const uint64_t now = global_timer_ns();
+                if (t0 == 0)
+                    t0 = now;
+                if (*abort) {
+                    cache = kGateFailed;
+                    break;
+                }
+                if ((int64_t)(now - t0) > timeout_ns) {
+                    *abort = 1u;
+                    record_error(status, kErrTimeout);
+                    cache = kGateFailed;
+                    break;
+                }
+            }
+        }
+    }
+    return __shfl_sync(0xffffffffu, cache, 0);
+}
+
+__device__ __forceinline__ int slot_gate_gm(const KernelArgs &a, const Shared &sh, const SlotRef &sr, uint32_t &cache)
+{
+    cache = slot_gate_wait_gm(sr.need, a.g_ctrl + sr.unit, a.epoch, cache, sh.abort, a.timeout_ns, a.device_status);
+    return cache == kGateFailed ? -1 : ((cache & kStopBit) ? 0 : 1);
+}
+
+// After the lanes' plain stores of a block state into the workspace: the
+// state becomes visible before its ready tag (lane 0 orders the warp's stores
+// it has synchronised with, then releases the tag).
+__device__ __forceinline__ void gm_publish(const SlotRef &sr)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence();
+        st_release_gpu_u64(sr.gflag, sr.tag);
+    }
 }
 
 // Bytes one block state occupies in a slot: flag word, m and l per head,
@@ -679,7 +761,9 @@ struct CudaEngine {
 // Tensor-core engine (bf16): S^T = K q^T with mma.m16n8k16 (tokens x heads),
 // then O^T = V^T P^T with P kept to ~16 significant bits as a bf16 hi + lo pair
 // (for G <= 4 both halves share one n8 tile: columns 0-3 hi, 4-7 lo).
-template <int D, int PAGE, int GMAX>
+// SINK: 0 pushes block states into the cluster leader's shared memory, 1
+// writes them into the workspace in global memory
+template <int D, int PAGE, int GMAX, int SINK = 0>
 struct MmaEngine {
     static constexpr int MT = PAGE / 16;  // token tiles
     static constexpr int KS = D / 16;     // head-dim tiles
@@ -865,9 +949,37 @@ struct MmaEngine {
         // slot layout of this engine: 16-byte vectors, vector (dt, r, c) holds
         // u[gA][d], u[gA+1][d], u[gA][d+8], u[gA+1][d+8] with d = 16 dt + r
         if (sr.need) {
-            const int g = slot_gate(a, sh, sr, gcache);
+            const int g = SINK ? slot_gate_gm(a, sh, sr, gcache) : slot_gate(a, sh, sr, gcache);
             if (g <= 0)
                 return g == 0;
+        }
+        if constexpr (SINK == 1) {
+            float *gs = sr.gslot;
+            if (lane == 0)
+                reinterpret_cast<uint32_t *>(gs)[0] = 0u;
+            if (writer) {
+                const bool w0 = gA < a.G, w1 = gA + 1 < a.G;
+                const float inv0 = (w0 && l2[0] > 0.f) ? rcp_approx(l2[0]) : 0.f;
+                const float inv1 = (w1 && l2[1] > 0.f) ? rcp_approx(l2[1]) : 0.f;
+                if (r == 0) {
+                    if (w0) {
+                        gs[4 + gA] = m2[0];
+                        gs[4 + GMAX + gA] = l2[0];
+                    }
+                    if (w1) {
+                        gs[4 + gA + 1] = m2[1];
+                        gs[4 + GMAX + gA + 1] = l2[1];
+                    }
+                }
+                constexpr int WPT = kShared ? 16 : 32;
+                const int widx = kShared ? (r * 2 + c) : (r * 4 + c);
+#pragma unroll
+                for (int dt = 0; dt < KS; ++dt)
+                    *reinterpret_cast<float4 *>(gs + u_off + 4 * (dt * WPT + widx)) =
+                        make_float4(tot[dt][0] * inv0, tot[dt][1] * inv1, tot[dt][2] * inv0, tot[dt][3] * inv1);
+            }
+            gm_publish(sr);
+            return true;
         }
         if (lane == 0) {
             mbar_arrive_expect_tx_cluster(sr.ready, slot_tx_bytes(a.G, D, GMAX, kEngineMma));
@@ -898,17 +1010,19 @@ struct MmaEngine {
     }
 };
 
-template <typename T, int D, int PAGE, int GMAX, int ENGINE>
-using EngineFor = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX>,
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, int SINK = 0>
+using EngineFor = typename std::conditional<ENGINE == kEngineMma, MmaEngine<D, PAGE, GMAX, SINK>,
                                             CudaEngine<T, D, PAGE, GMAX>>::type;
 
 // eng holds the unit's queries, loaded before the set-up barriers.  GATE:
 // the window reaches past the state ring, so a finished state waits for its
-// slot (slot_gate).
-template <typename T, int D, int PAGE, int GMAX, int ENGINE, bool GATE = false>
+// slot (slot_gate).  SINK = 1: states go to the workspace ring (a.Rg slots
+// per unit, always gated).
+template <typename T, int D, int PAGE, int GMAX, int ENGINE, bool GATE = false, int SINK = 0>
 __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h, int cw,
-                             EngineFor<T, D, PAGE, GMAX, ENGINE> &eng)
+                             EngineFor<T, D, PAGE, GMAX, ENGINE, SINK> &eng)
 {
+    static_assert(SINK == 0 || ENGINE == kEngineMma, "the workspace sink is built for the tensor-core engine");
     const int lane = threadIdx.x & 31;
     float *pbuf = sh.pbuf + (ENGINE == kEngineMma ? 0 : cw * PAGE * GMAX);
     const uint32_t ring_cl = mapa(sh.ring_leader, 0);
@@ -924,21 +1038,38 @@ __device__ void compute_role(const KernelArgs &a, const Shared &sh, int b, int h
         if (j == kEndOfStream)
             break;
         const int nv = (int)sh.stage_nv[s];
-        const uint32_t slot = j % (uint32_t)a.R;
-        const uint32_t need = (GATE && j >= (uint32_t)a.R) ? j - (uint32_t)a.R + 1u : 0u;
-        SlotRef sr{ring_cl + slot * sh.L.slot_bytes, ready_cl + 8u * slot, need, ctrl_cl};
+        SlotRef sr;
+        if constexpr (SINK == 0) {
+            const uint32_t slot = j % (uint32_t)a.R;
+            sr.base = ring_cl + slot * sh.L.slot_bytes;
+            sr.ready = ready_cl + 8u * slot;
+            sr.need = (GATE && j >= (uint32_t)a.R) ? j - (uint32_t)a.R + 1u : 0u;
+            sr.ctrl = ctrl_cl;
+        } else {
+            const int unit = b * a.Hkv + h;
+            const uint32_t gslot = j % (uint32_t)a.Rg;
+            sr.unit = unit;
+            sr.gslot = a.g_states + ((int64_t)unit * a.Rg + gslot) * (sh.L.slot_bytes / 4);
+            sr.gflag = a.g_flags + (int64_t)unit * a.Rg + gslot;
+            sr.tag = ((unsigned long long)a.epoch << 32) | (unsigned long long)(j + 1u);
+            sr.need = j >= (uint32_t)a.Rg ? j - (uint32_t)a.Rg + 1u : 0u;
+        }
         if (nv < 0) {  // bad page: forward the flag, free the stage
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(sh.empty(s));
             if (sr.need) {
-                const int g = slot_gate(a, sh, sr, gcache);
+                const int g = SINK ? slot_gate_gm(a, sh, sr, gcache) : slot_gate(a, sh, sr, gcache);
                 if (g < 0)
                     break;
                 if (g == 0)
                     continue;
             }
-            if (lane == 0) {
+            if constexpr (SINK == 1) {
+                if (lane == 0)
+                    reinterpret_cast<uint32_t *>(sr.gslot)[0] = 1u;
+                gm_publish(sr);
+            } else if (lane == 0) {
                 mbar_arrive_expect_tx_cluster(sr.ready, 4u);
                 st_async_b32(sr.base, 1u, sr.ready);
             }
@@ -1924,8 +2055,10 @@ __device__ void merge_role_multi(const KernelArgs &a, const Shared &sh, int b, i
 
 // NQ: query tokens sharing the walk (1: merge_role, else merge_role_multi).
 // DET: false for the single-query walk without the detector (see merge_role).
+// (the shared walks with one merge warp launch at most eight warps: their
+// bound leaves them the registers the two-token merge needs)
 template <typename T, int D, int PAGE, int GMAX, int ENGINE, int NMW, int NQ = 1, bool DET = true>
-__global__ void __launch_bounds__(kMaxThreads, 1)
+__global__ void __launch_bounds__((NQ > 1 && NMW == 1) ? 256 : kMaxThreads, 1)
     art_walk_kernel(const KernelArgs a, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv)
 {

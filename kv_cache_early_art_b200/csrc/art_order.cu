@@ -229,12 +229,207 @@ struct ScoreArgs {
     float *scores;
     int64_t scs0;
     int B, Hq, Hkv, G, d, page, max_blocks, num_pages, blocks_per_warp;
+    int q_vec;                  // q rows may be read 4 channels at a time (aligned)
     float scale;
     int32_t *status;
 };
 
+// 16 raw bytes of a summary row (8 bf16 or 4 fp32 channels), unpacked at use
+template <typename TS>
+__device__ __forceinline__ uint4 raw16(const TS *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+template <typename TS>
+__device__ __forceinline__ void unpack16(const uint4 &v, float *f)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (std::is_same<TS, float>::value) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            f[i] = __uint_as_float(w[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+}
+
+// The query rows' group sums for 4 consecutive channels of head h:
+// sum over g < G of q[h G + g][c .. c + 3] (fp32, in head order).
+template <typename TQ>
+__device__ __forceinline__ void group_sum4(const TQ *qb, int64_t qs1, int h, int G, int c, bool vec, float (&s)[4])
+{
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        s[e] = 0.f;
+    for (int g0 = 0; g0 < G; g0 += 4) {
+        // four rows' reads in flight before any is added
+        float f[4][4];
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                f[gg][e] = 0.f;
+            if (g0 + gg < G) {
+                const TQ *row = qb + (int64_t)(h * G + g0 + gg) * qs1 + c;
+                if (vec) {
+                    if constexpr (std::is_same<TQ, float>::value) {
+                        const float4 v = __ldg(reinterpret_cast<const float4 *>(row));
+                        f[gg][0] = v.x; f[gg][1] = v.y; f[gg][2] = v.z; f[gg][3] = v.w;
+                    } else {
+                        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(row));
+                        f[gg][0] = __uint_as_float(v.x << 16);
+                        f[gg][1] = __uint_as_float(v.x & 0xffff0000u);
+                        f[gg][2] = __uint_as_float(v.y << 16);
+                        f[gg][3] = __uint_as_float(v.y & 0xffff0000u);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        f[gg][e] = Vec<TQ>::scalar(row + e);
+                }
+            }
+        }
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg)
+            if (g0 + gg < G)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    s[e] += f[gg][e];
+    }
+}
+
+// One warp scores NBW consecutive blocks of one sequence, two at a time
+// (CH summary vectors of VE channels per lane and block).  The group sums of
+// the query rows sit in shared memory, filled once per CTA; the page indices
+// and the first pair's summaries are requested before that prologue, so its
+// reads overlap theirs, and each later pair's summaries are requested while
+// the previous pair is multiplied.  The arithmetic (group sums in head order,
+// products vector by vector, a five-level butterfly) is fixed, so the scores
+// are reproducible bit for bit.
 template <typename TQ, typename TS, int CH>
-__global__ void __launch_bounds__(kThreads) art_block_score_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kThreads, CH <= 2 ? 4 : 2) art_block_score_kernel(ScoreArgs a)
+{
+    extern __shared__ float qg[];   // [Hkv * d]: sum of the group's query heads
+    constexpr int VE = Vec<TS>::E;
+    // the rank kernel may launch now; its griddepcontrol.wait holds it until
+    // this whole grid has finished and its stores are visible
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NBW = a.blocks_per_warp;                // even, at most 32
+    const int jw = (blockIdx.x * kWarps + warp) * NBW;
+    const int L = a.sl[b];
+    int pidx = -1;
+    if (lane < NBW && jw + lane < a.max_blocks)
+        pidx = a.pt[(int64_t)b * a.pts0 + jw + lane];
+    const int VR = a.d / VE;
+    const int nv = a.Hkv * a.d / VE;                  // vectors per summary
+    const int N = min(n_blocks_of(L, a.page), a.max_blocks);
+    const TS *sb = static_cast<const TS *>(a.sum);
+    // summaries of the pair starting at block jw + k (zeros where absent)
+    auto fetch = [&](int k, uint4 (&ra)[CH], uint4 (&rb)[CH], bool &va, bool &vb) {
+        const int ja = jw + k, jb = ja + 1;
+        const int pa = __shfl_sync(0xffffffffu, pidx, k & 31);
+        const int pbk = __shfl_sync(0xffffffffu, pidx, (k + 1) & 31);
+        va = ja < N && pa >= 0 && pa < a.num_pages;
+        vb = jb < N && pbk >= 0 && pbk < a.num_pages;
+        const TS *ba = sb + (int64_t)(va ? pa : 0) * a.ss0;
+        const TS *bbp = sb + (int64_t)(vb ? pbk : 0) * a.ss0;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int v = lane + 32 * c;
+            const int h = v / VR, cv = v - h * VR;
+            const int64_t off = (int64_t)h * a.ss1 + cv * VE;
+            ra[c] = make_uint4(0u, 0u, 0u, 0u);
+            rb[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (v < nv && va)
+                ra[c] = raw16<TS>(ba + off);
+            if (v < nv && vb)
+                rb[c] = raw16<TS>(bbp + off);
+        }
+    };
+    uint4 ca[CH], cb[CH];
+    bool cva = false, cvb = false;
+    if (jw < a.max_blocks)
+        fetch(0, ca, cb, cva, cvb);   // in flight during the prologue below
+    const int HD = a.Hkv * a.d;
+    const TQ *qb = static_cast<const TQ *>(a.q) + (int64_t)b * a.qs0;
+    for (int i4 = threadIdx.x; i4 < HD / 4; i4 += kThreads) {
+        const int idx = i4 * 4, h = idx / a.d, c = idx - h * a.d;
+        float sum4[4];
+        group_sum4<TQ>(qb, a.qs1, h, a.G, c, a.q_vec != 0, sum4);
+        *reinterpret_cast<float4 *>(qg + idx) = make_float4(sum4[0], sum4[1], sum4[2], sum4[3]);
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && threadIdx.x == 0 && n_blocks_of(L, a.page) > a.max_blocks)
+        report(a.status, ART_ERR_BAD_INDEX);
+    if (jw >= a.max_blocks)
+        return;                                       // no barrier follows
+    float *srow = a.scores + (int64_t)b * a.scs0;
+    for (int k = 0; k < NBW; k += 2) {
+        const int ja = jw + k, jb = ja + 1;
+        if (ja >= a.max_blocks)
+            break;
+        uint4 na[CH], nb2[CH];
+        bool nva = false, nvb = false;
+        if (k + 2 < NBW && ja + 2 < a.max_blocks)
+            fetch(k + 2, na, nb2, nva, nvb);
+        float acc_a = 0.f, acc_b = 0.f;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int v = lane + 32 * c;
+            if (v < nv) {
+                const int h = v / VR, cv = v - h * VR;
+                const float *qv = qg + h * a.d + cv * VE;
+                float fa[VE], fb[VE];
+                unpack16<TS>(ca[c], fa);
+                unpack16<TS>(cb[c], fb);
+#pragma unroll
+                for (int e = 0; e < VE; ++e) {
+                    acc_a = fmaf(qv[e], fa[e], acc_a);
+                    acc_b = fmaf(qv[e], fb[e], acc_b);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            acc_a += __shfl_xor_sync(0xffffffffu, acc_a, o);
+            acc_b += __shfl_xor_sync(0xffffffffu, acc_b, o);
+        }
+        if (lane == 0) {
+            const float nan = __int_as_float(0x7fc00000);
+            float sa = ja >= N ? -INFINITY : (cva ? acc_a * a.scale : nan);
+            if (sa == 0.f)
+                sa = 0.f;   // -0 is stored as +0
+            srow[ja] = sa;
+            if ((ja < N && !cva) || (jb < N && !cvb))
+                report(a.status, ART_ERR_BAD_INDEX);
+            if (jb < a.max_blocks) {
+                float sbv = jb >= N ? -INFINITY : (cvb ? acc_b * a.scale : nan);
+                if (sbv == 0.f)
+                    sbv = 0.f;
+                srow[jb] = sbv;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            ca[c] = na[c];
+            cb[c] = nb2[c];
+        }
+        cva = nva;
+        cvb = nvb;
+    }
+}
+
+// Wide summaries (more than four vectors per lane): the group sums of the
+// query rows sit in shared memory, filled by the whole CTA first.
+template <typename TQ, typename TS, int CH>
+__global__ void __launch_bounds__(kThreads) art_block_score_wide_kernel(ScoreArgs a)
 {
     // CH: summary vectors per lane and block kept in flight (1, 2 or 4)
     extern __shared__ float qg[];   // [Hkv * d]: sum of the group's query heads
@@ -481,6 +676,19 @@ cudaError_t launch_score_ch(const ScoreArgs &a, dim3 grid, size_t smem, cudaStre
     return cudaSuccess;
 }
 
+template <typename TQ, typename TS>
+cudaError_t launch_score_wide(const ScoreArgs &a, dim3 grid, size_t smem, cudaStream_t s)
+{
+    auto fn = art_block_score_wide_kernel<TQ, TS, 4>;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    fn<<<grid, kThreads, smem, s>>>(a);
+    return cudaSuccess;
+}
+
 // loads in flight per lane and block: just enough to cover one summary
 template <typename TQ, typename TS>
 cudaError_t launch_score(const ScoreArgs &a, dim3 grid, size_t smem, cudaStream_t s)
@@ -490,7 +698,9 @@ cudaError_t launch_score(const ScoreArgs &a, dim3 grid, size_t smem, cudaStream_
         return launch_score_ch<TQ, TS, 1>(a, grid, smem, s);
     if (per_lane == 2)
         return launch_score_ch<TQ, TS, 2>(a, grid, smem, s);
-    return launch_score_ch<TQ, TS, 4>(a, grid, smem, s);
+    if (per_lane <= 4)
+        return launch_score_ch<TQ, TS, 4>(a, grid, smem, s);
+    return launch_score_wide<TQ, TS>(a, grid, smem, s);
 }
 
 }  // namespace
@@ -612,6 +822,11 @@ art_status_t art_build_order_importance(const art_tensor_t *q, const art_tensor_
     a.num_pages = (int)NP;
     a.scale = sm_scale > 0.f ? sm_scale : (float)(1.0 / std::sqrt((double)d));
     a.status = device_status;
+    {
+        // four channels per load where every q row starts on such a boundary
+        const int64_t es = elem_size(q->dtype), vb = 4 * es;
+        a.q_vec = aligned(q->data, (uintptr_t)vb) && (q->stride[0] * es) % vb == 0 && (q->stride[1] * es) % vb == 0;
+    }
     // about four CTAs per SM over the whole batch; an even number of blocks per warp, at most 32
     const int64_t warps = (int64_t)sm_count() * 4 * kWarps;
     int64_t nbw = (B * mb + warps - 1) / warps;

@@ -23,6 +23,8 @@ KernelFn bf16_cuda(int gmax, int d, int page);
 KernelFn bf16_mma(int gmax, int nmw, int d, int page, bool detector);
 // bf16 caches, tensor-core block engine, dedicated merge CTA (gmax 4 or 8)
 KernelFn bf16_mma_dl(int gmax, int d, int page, bool detector);
+// the same merge reached through a workspace (no clusters, cooperative launch)
+KernelFn bf16_mma_gr(int gmax, int d, int page, bool detector);
 // two query tokens sharing one walk (head dim 128)
 KernelFn multi(bool f32, int engine, int page, int gmax, int nmw);
 

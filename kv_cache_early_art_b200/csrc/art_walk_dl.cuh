@@ -51,7 +51,7 @@ constexpr int kDLCtlOff = kDLSumFloats + 2 * kDLBetaFloats;
 constexpr int kDLRedFloats = kDLCtlOff + 16;
 constexpr int kDLNone = 0x7fffffff;  // no final decision published yet
 constexpr int kDLFailed = -1;
-constexpr int kDLBars = 8;           // sums_full[2], beta_full[2], beta_empty[2], dec[2]
+constexpr int kDLBars = 10;          // sums_full[2], beta_full[2], beta_empty[2], dec[2], landed[2]
 
 // Shared-memory carve-up.  The control words and the state ring's ready
 // barriers sit at the same offsets in every CTA of the cluster, so the workers
@@ -99,6 +99,7 @@ struct DLBars {
     uint32_t beta_full;   // the shares of a batch are written (count 1)
     uint32_t beta_empty;  // the fold warps have read them (count NMF)
     uint32_t dec;         // the decision warp has decided a batch (count 1)
+    uint32_t landed;      // a batch's states have been copied in from the workspace (count 1)
 };
 
 // Bounded wait of a whole warp until pred() holds for lane 0's view.
@@ -508,9 +509,13 @@ __device__ void fold_role_dl(const KernelArgs &a, const Shared &sh, int b, int h
 
 // ---- decision warp ----------------------------------------------------------------
 
-template <int D, int GMAX, int ENGINE, int NMF, bool DET>
+// GM: publish the merged count and the stop in the workspace (the fetching
+// CTAs are not in this CTA's cluster) instead of this CTA's shared memory.
+template <int D, int GMAX, int ENGINE, int NMF, bool DET, bool GM = false>
 __device__ void decide_role_dl(const KernelArgs &a, const Shared &sh, int b, int h, int N, const DLBars &bars)
 {
+    const unsigned long long ep = (unsigned long long)a.epoch << 32;
+    unsigned long long *gctrl = GM ? a.g_ctrl + (b * a.Hkv + h) : nullptr;
     const int lane = threadIdx.x & 31;
     const float eps_m = a.eps_m_arr ? a.eps_m_arr[b] : a.eps_m;
     const float eps_d = a.eps_d_arr ? a.eps_d_arr[b] : a.eps_d;
@@ -591,7 +596,10 @@ __device__ void decide_role_dl(const KernelArgs &a, const Shared &sh, int b, int
         ++batch;
         if (lane == 0) {
             // batch decided without a stop: its slots go back to the producers
-            st_release_cluster_u32(ctrl_cl, (uint32_t)j0);
+            if constexpr (GM)
+                st_release_gpu_u64(gctrl, ep | (uint32_t)j0);
+            else
+                st_release_cluster_u32(ctrl_cl, (uint32_t)j0);
             if (j0 >= N)
                 ctl[3] = N;  // the walk is over (before the arrive: the fold warps read it after their wait)
             mbar_arrive(bars.dec + 8u * e);
@@ -602,7 +610,10 @@ __device__ void decide_role_dl(const KernelArgs &a, const Shared &sh, int b, int
     if (lane == 0) {
         if (failed)
             ctl[3] = kDLFailed;
-        st_release_cluster_u32(ctrl_cl, kStopBit | (failed ? 0u : (uint32_t)stop));
+        if constexpr (GM)
+            st_release_gpu_u64(gctrl, ep | kStopBit | (failed ? 0u : (uint32_t)stop));
+        else
+            st_release_cluster_u32(ctrl_cl, kStopBit | (failed ? 0u : (uint32_t)stop));
         a.stop_block[(int64_t)b * a.stop_sb + (int64_t)h * a.stop_sh] = failed ? -1 : stop;
     }
 }
@@ -657,6 +668,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     bars.beta_full = bars.sums_full + 16u;
     bars.beta_empty = bars.sums_full + 32u;
     bars.dec = bars.sums_full + 48u;
+    bars.landed = bars.sums_full + 64u;
     sh.ring_leader = smem_u32(base + LL.ring_off);
     sh.ready_leader = sh.bar_ready;
     volatile int *ctl = reinterpret_cast<volatile int *>(sh.red + kDLCtlOff);
@@ -709,7 +721,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                 fold_role_dl<D, GMAX, ENGINE, NMF, DET>(a, sh, b, h, N, warp - 2, bars);
         } else {
             if (warp == 0)
-                producer_role<T, D, PAGE, ENGINE, true>(a, sh, &tmk, &tmv, b, h, N, Lseq, (uint32_t)wrank, W,
+                producer_role<T, D, PAGE, ENGINE, 1>(a, sh, &tmk, &tmv, b, h, N, Lseq, (uint32_t)wrank, W,
                                                          first_lb, first_pp);
             else if (warp <= a.NW)
                 compute_role<T, D, PAGE, GMAX, ENGINE, true>(a, sh, b, h, warp - 1, eng);

@@ -2,6 +2,7 @@
 // tensor-core block engine.
 #include "art_walk.h"
 #include "art_walk_dl.cuh"
+#include "art_walk_gr.cuh"
 
 namespace art_walk {
 
@@ -47,6 +48,18 @@ KernelFn bf16_mma_dl(int gmax, int d, int page, bool detector)
     if (detector)
         return gmax == 4 ? art_walk_dl_kernel<T, 128, 64, 4, E, 4, true> : art_walk_dl_kernel<T, 128, 64, 8, E, 8, true>;
     return gmax == 4 ? art_walk_dl_kernel<T, 128, 64, 4, E, 4, false> : art_walk_dl_kernel<T, 128, 64, 8, E, 8, false>;
+}
+
+KernelFn bf16_mma_gr(int gmax, int d, int page, bool detector)
+{
+    using art::art_walk_gr_kernel;
+    using T = __nv_bfloat16;
+    constexpr int E = art::kEngineMma;
+    if (d != 128 || page != 64)
+        return nullptr;
+    if (detector)
+        return gmax == 4 ? art_walk_gr_kernel<T, 128, 64, 4, E, 4, true> : art_walk_gr_kernel<T, 128, 64, 8, E, 8, true>;
+    return gmax == 4 ? art_walk_gr_kernel<T, 128, 64, 4, E, 4, false> : art_walk_gr_kernel<T, 128, 64, 8, E, 8, false>;
 }
 
 }  // namespace art_walk

@@ -138,7 +138,7 @@ def test_ex_option_errors(art):
     for field, val in (("engine", 3), ("cluster_size", 17), ("stages", 9), ("stages", 1), ("window", 129),
                        ("compute_warps", 7), ("window", 7), ("debug_flags", 2), ("timeout_ns", -1),
                        ("prefetch", -2), ("prefetch", 65), ("detector_off", 2), ("detector_off", -1),
-                       ("merge_cta", 2), ("merge_cta", -2)):
+                       ("merge_cta", 3), ("merge_cta", -2), ("workspace_bytes", -1)):
         setattr(p, field, val)
         assert lib.art_decode_attention_ex(ctypes.byref(p), None) == -5, field
         setattr(p, field, 0)
