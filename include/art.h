@@ -69,7 +69,9 @@ typedef enum {
     ART_ERR_PARAM = -5,          /* eps < 0 or NaN, P < 0, min_blocks < 0, bad option    */
     ART_ERR_LAUNCH = -6,         /* the CUDA runtime refused the launch                  */
     ART_ERR_DEVICE_TIMEOUT = -7, /* (device_status) a bounded wait expired               */
-    ART_ERR_BAD_INDEX = -8       /* (device_status) order/page entry or length invalid   */
+    ART_ERR_BAD_INDEX = -8,      /* (device_status) order/page entry or length invalid   */
+    ART_ERR_SCRATCH_SIZE = -9    /* art_decode_attention_no_alloc: the problem needs     */
+                                 /* more than ART_NO_ALLOC_SCRATCH_BYTES of scratch      */
 } art_status_t;
 
 /*
@@ -204,6 +206,44 @@ art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
  * invalid.  Nothing is launched.
  */
 int64_t art_workspace_bytes(const art_params_t *p);
+
+/*
+ * art_decode_attention_no_alloc -- art_decode_attention_ex with merge_cta = 2
+ * (one merge CTA and several fetching CTAs per unit, the block states handed
+ * over through scratch memory), but the scratch is a fixed device array inside
+ * this library, so the call allocates nothing.  The paper has no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc: a serving
+ * engine whose memory pool has already claimed nearly all device memory (a
+ * cudaMalloc there fails or steals from the pool), a latency-bound decode loop
+ * that may not stall on an allocation (cudaMalloc and cudaFree can block the
+ * host and synchronise the device), or a plug-in that may not grow the device
+ * footprint of the application hosting it.
+ *
+ *  p           as for art_decode_attention_ex, except: workspace NULL and
+ *              workspace_bytes 0 (else ART_ERR_PARAM), merge_cta 0 or 2
+ *              (else ART_ERR_PARAM).  The caller still owns and passes every
+ *              input and output tensor.
+ *  Returns     ART_ERR_SCRATCH_SIZE when the problem needs more scratch than
+ *              ART_NO_ALLOC_SCRATCH_BYTES even with the smallest ring (16
+ *              block states per unit; about 67 KB per unit with 8 query heads
+ *              per kv head, so about 60 units), ART_ERR_UNSUPPORTED where the
+ *              workspace walk is not built (BF16 caches on the tensor-core
+ *              engine, d = 128, 64-token pages, one query token, every CTA
+ *              resident at once), otherwise what art_decode_attention_ex
+ *              returns.  The ring is the largest that fits the array.
+ *
+ * The array (ART_NO_ALLOC_SCRATCH_BYTES, 256-byte aligned) is held by every
+ * GPU on which the library's device code is loaded, until the process exits.
+ * The first call on each device looks up the array's device address with that
+ * device current and keeps it; make that first call before any stream capture
+ * begins.  Every call on a device shares the one array and it keeps what the
+ * last call left; nothing in it needs clearing, since each control word the
+ * walk reads is tagged with the call that wrote it.  Calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on the array:
+ * order them on one stream or serialise them.
+ */
+#define ART_NO_ALLOC_SCRATCH_BYTES (4 << 20)
+art_status_t art_decode_attention_no_alloc(const art_params_t *p, art_stream_t stream);
 
 /*
  * art_decode_attention_multi -- n_queries query tokens of each sequence (for

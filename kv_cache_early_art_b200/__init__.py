@@ -12,7 +12,7 @@ _BINDING_NAMES = {
     "art_decode_attention", "art_decode_attention_ex", "art_decode_attention_multi",
     "art_build_order_sink_recency", "art_strerror",
     "art_page_summary", "art_build_order_importance",
-    "art_version", "art_workspace_bytes", "ArtError", "descriptor", "raw_library", "ENGINE_AUTO", "ENGINE_CUDA", "ENGINE_MMA",
+    "art_version", "art_workspace_bytes", "art_decode_attention_no_alloc", "ArtError", "descriptor", "raw_library", "ENGINE_AUTO", "ENGINE_CUDA", "ENGINE_MMA",
     "STATUS", "ArtParams", "ArtTensor", "ArtLaunchInfo", "LIB_PATH",
 }
 

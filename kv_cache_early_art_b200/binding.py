@@ -29,6 +29,7 @@ _DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.int32: I32}
 STATUS = {
     0: "ART_OK", -1: "ART_ERR_NULL", -2: "ART_ERR_SHAPE", -3: "ART_ERR_DTYPE", -4: "ART_ERR_UNSUPPORTED",
     -5: "ART_ERR_PARAM", -6: "ART_ERR_LAUNCH", -7: "ART_ERR_DEVICE_TIMEOUT", -8: "ART_ERR_BAD_INDEX",
+    -9: "ART_ERR_SCRATCH_SIZE",
 }
 ENGINE_AUTO, ENGINE_CUDA, ENGINE_MMA = 0, 1, 2
 
@@ -80,6 +81,8 @@ _lib.art_build_order_importance.argtypes = [_P(ArtTensor)] * 4 + [ctypes.c_int32
 _lib.art_build_order_importance.restype = ctypes.c_int
 _lib.art_workspace_bytes.argtypes = [_P(ArtParams)]
 _lib.art_workspace_bytes.restype = ctypes.c_int64
+_lib.art_decode_attention_no_alloc.argtypes = [_P(ArtParams), ctypes.c_void_p]
+_lib.art_decode_attention_no_alloc.restype = ctypes.c_int
 _lib.art_strerror.argtypes = [ctypes.c_int]
 _lib.art_strerror.restype = ctypes.c_char_p
 _lib.art_version.argtypes = []
@@ -258,6 +261,32 @@ def art_workspace_bytes(q, k_cache, v_cache, page_table, block_order, seq_lens, 
     if n < 0:
         raise ArtError(n, "art_workspace_bytes")
     return n
+
+
+def art_decode_attention_no_alloc(q, k_cache, v_cache, page_table, block_order, seq_lens, *, eps_m=0.0, eps_d=0.0,
+                                  P=0, min_blocks=0, sm_scale=0.0, eps_m_per_seq=None, eps_d_per_seq=None,
+                                  P_per_seq=None, min_blocks_per_seq=None, blocks_fetched=None, device_status=None,
+                                  engine=0, cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0,
+                                  prefetch=0, detector_off=0, out=None, stop_block=None, stream=None,
+                                  want_info=False):
+    """art_decode_attention_no_alloc in art.h: the workspace walk with the
+    library's own fixed scratch array, for callers that cannot allocate
+    device memory (pass out and stop_block to allocate nothing here either).
+    Returns (out, stop_block) or those plus the launch info dict."""
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if stop_block is None:
+        stop_block = torch.empty(B, k_cache.shape[1], dtype=torch.int32, device=q.device)
+    p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
+                      min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
+                      blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
+                      timeout_ns, 0, prefetch, detector_off, 0)
+    st = _lib.art_decode_attention_no_alloc(ctypes.byref(p), _stream(stream))
+    _check(st, "art_decode_attention_no_alloc")
+    if want_info:
+        return out, stop_block, info.as_dict()
+    return out, stop_block
 
 
 def art_build_order_sink_recency(seq_lens, page, block_order=None, max_blocks=None, stream=None):

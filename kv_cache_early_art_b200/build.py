@@ -14,8 +14,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libart.so")
 # one translation unit per group of walk instantiations, so that they compile in parallel
 SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu", "art_order.cu", "art_walk_f32.cu", "art_walk_bf16.cu",
-                                           "art_walk_mma.cu", "art_walk_multi.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh", "art_host.h", "art_walk.h", "art_walk_dl.cuh")] + [
+                                           "art_walk_mma.cu", "art_walk_multi.cu", "art_no_alloc.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("art_kernels.cuh", "art_ptx.cuh", "art_host.h", "art_walk.h", "art_walk_dl.cuh", "art_walk_gr.cuh")] + [
     os.path.join(ROOT, "include", "art.h")]
 
 NVCC_FLAGS = [

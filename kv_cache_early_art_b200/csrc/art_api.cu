@@ -835,6 +835,41 @@ art_status_t launch(const art_params_t *p, art_stream_t stream, int nq = 1, bool
 
 }  // namespace
 
+namespace art_host {
+
+int64_t gr_min_workspace_bytes(const art_params_t *p)
+{
+    if (!p)
+        return ART_ERR_NULL;
+    Problem pr;
+    art_status_t st = check_tensors(p, &pr);
+    if (st != ART_OK)
+        return st;
+    if ((st = check_params(p)) != ART_OK)
+        return st;
+    DeviceInfo di;
+    if ((st = device_info(&di)) != ART_OK)
+        return st;
+    // any non-null workspace without a size limit: choose_gr then settles the
+    // launch shape (it never dereferences the pointer)
+    art_params_t q = *p;
+    q.merge_cta = 2;
+    q.workspace = reinterpret_cast<void *>(static_cast<uintptr_t>(256));
+    q.workspace_bytes = INT64_MAX;
+    Shape s;
+    bool chosen = false;
+    int64_t need = 0;
+    if ((st = choose_gr(&q, pr, di, &s, &chosen, &need)) != ART_OK)
+        return st;
+    if (!chosen)
+        return 0;
+    const uint32_t slot =
+        art::make_dl_layout(0, s.R, pr.page, pr.d, (int)elem_size(pr.dtype), s.gmax, s.R).slot_bytes;
+    return art::gr_workspace_bytes(pr.B * pr.Hkv, s.W, 16, slot);
+}
+
+}  // namespace art_host
+
 extern "C" {
 
 art_status_t art_decode_attention_ex(const art_params_t *p, art_stream_t stream)
@@ -945,6 +980,7 @@ const char *art_strerror(art_status_t s)
     case ART_ERR_LAUNCH: return "the CUDA runtime refused the launch";
     case ART_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
     case ART_ERR_BAD_INDEX: return "an order or page-table entry, or a sequence length, is out of range";
+    case ART_ERR_SCRATCH_SIZE: return "the problem needs more scratch memory than the library's fixed array holds";
     }
     return "unknown status";
 }

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(art):
 
 
 def test_strerror_and_version(art):
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         s = art.art_strerror(code)
         assert s and s != "unknown status"
     assert art.art_strerror(-99) == "unknown status"
