@@ -85,7 +85,11 @@ typedef enum {
  *  page_table  [B, max_blocks] I32: physical page of logical block lb of sequence b.
  *  block_order [B, max_blocks] I32: logical block visited at walk step j; entries
  *                                   0..N_b-1 must be a permutation of 0..N_b-1 where
- *                                   N_b = ceil(seq_lens[b] / page).  Entries past
+ *                                   N_b = ceil(seq_lens[b] / page).  An entry out
+ *                                   of [0, N_b) is reported (ART_ERR_BAD_INDEX); a
+ *                                   repeated or missing block is not detected (the
+ *                                   walk would fold one block twice and skip
+ *                                   another: the result is undefined).  Entries past
  *                                   N_b are never read.  May be NULL (or have NULL
  *                                   data): the walk then takes the default order
  *                                   [0, N_b-1, ..., 1] (sink block, then newest to

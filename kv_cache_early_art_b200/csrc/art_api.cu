@@ -564,10 +564,13 @@ art_status_t choose_dl(const art_params_t *p, const Problem &pr, const DeviceInf
             return ART_OK;
     }
     s.C = C;
-    // the window reaches past the ring by the pages the fetching CTAs can hold
-    // in their stages: those are fetched and computed while the merge still
-    // holds every slot, and their states wait for a slot (slot_gate)
-    s.RF = p->window ? p->window : s.R + (C - 1) * s.S;
+    // the window reaches past the ring by two merge batches (at most the pages
+    // the fetching CTAs can hold in their stages): those are fetched and
+    // computed while the merge still holds every slot, and their states wait
+    // for a slot (slot_gate).  A deeper window read more pages past the stop
+    // on the few-unit workloads without a faster walk.
+    const int past = (C - 1) * s.S < 16 ? (C - 1) * s.S : 16;
+    s.RF = p->window ? p->window : s.R + past;
     s.RF = s.RF > 128 ? 128 : s.RF;
     if (s.RF < s.R)
         s.RF = s.R;

@@ -7,7 +7,7 @@ import bench
 SOURCES = ("kv_cache_early_art_b200/csrc/art_kernels.cuh", "kv_cache_early_art_b200/csrc/art_ptx.cuh",
            "kv_cache_early_art_b200/csrc/art_api.cu", "kv_cache_early_art_b200/csrc/art_host.h",
            "kv_cache_early_art_b200/build.py", "kv_cache_early_art_b200/csrc/art_walk.h",
-           "kv_cache_early_art_b200/csrc/art_walk_dl.cuh",
+           "kv_cache_early_art_b200/csrc/art_walk_dl.cuh", "kv_cache_early_art_b200/csrc/art_walk_gr.cuh",
            "kv_cache_early_art_b200/csrc/art_walk_f32.cu", "kv_cache_early_art_b200/csrc/art_walk_bf16.cu",
            "kv_cache_early_art_b200/csrc/art_walk_mma.cu", "kv_cache_early_art_b200/csrc/art_walk_multi.cu")
 
