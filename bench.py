@@ -309,7 +309,8 @@ def run_ours(args):
     import kv_cache_early_art_b200 as art
     from kv_cache_early_art_b200.workloads import make_workload
 
-    w = make_workload(args.workload, seed=replica_seed(rank), device=dev)
+    w = make_workload(args.workload, seed=replica_seed(rank), device=dev, seq_len=args.seq_len)
+    wname = w.name
     B, Hkv, page, d = w.B, w.Hkv, w.page, w.d
     esize = w.k_cache.element_size()
     N = w.n_blocks().to(dev)
@@ -404,7 +405,7 @@ def run_ours(args):
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (ms_walk / 1000.0) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "traffic": ncu_traffic(args.workload if T == 1 else f"{args.workload}_shared{T}"),
+            "traffic": ncu_traffic(wname if T == 1 else f"{wname}_shared{T}"),
             "peak_kind": peak_kind,
             "kernel": "art_walk_kernel (the whole step: the order is built inside it)" if T == 1 else
                       f"art_walk_kernel, {T} tokens per walk (the whole step)",
@@ -413,7 +414,7 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": str(w.k_cache.dtype).replace("torch.", "").replace("bfloat16", "bf16"),
-            "data": "synthetic", "config": dict(config_for(args.workload, w, ws), **(
+            "data": "synthetic", "config": dict(config_for(wname, w, ws), **(
                 {"queries_per_sequence": T, "queries": "draft tokens sharing one walk: token 0 the workload's "
                  "query, token 1 that query plus 0.5 N(0,1); each token keeps its own ART decision"}
                 if T > 1 else {})),
@@ -489,7 +490,7 @@ def run_ours(args):
         qps, cores, nseq, el = time_oracle(w_cpu, args.cpu_seconds)
         qps1, _, nseq1, el1 = time_oracle(w_cpu, args.cpu_seconds / 2, ncores=1)
         line["cpu_baseline"] = {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                                "sample": f"{nseq} {args.workload} sequences (decode queries, every kv head), "
+                                "sample": f"{nseq} {wname} sequences (decode queries, every kv head), "
                                           f"cycling through the batch, in {el:.1f} s",
                                 "one_core": {"value": qps1, "sample": f"{nseq1} sequences in {el1:.1f} s"}}
     if ws > 1:
@@ -694,6 +695,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="replace a uniform-length workload's length (a smaller case of the same launch, "
+                         "for profiling); the line then names <workload>_L<len>")
     ap.add_argument("--multi", type=int, default=1, choices=[1, 2],
                     help="decode tokens per sequence sharing one walk (2: art_decode_attention_multi)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

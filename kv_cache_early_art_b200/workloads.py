@@ -288,10 +288,17 @@ def make_custom(*, B, Hq, Hkv, d, page, dtype="bf16", seq_lens, seed=0, keys="re
                     dict(planted_pos=planted_pos, seed=seed, dtype=dtype))
 
 
-def make_workload(name: str, seed: int = 0, device="cpu") -> Workload:
-    """Build one of the named workloads in ``CONFIGS``."""
+def make_workload(name: str, seed: int = 0, device="cpu", seq_len: Optional[int] = None) -> Workload:
+    """Build one of the named workloads in ``CONFIGS``.  seq_len replaces the
+    length of a uniform-length workload (a smaller case of the same shape,
+    e.g. for profiling); the workload is then named ``<name>_L<seq_len>``."""
     c = dict(CONFIGS[name])
     B = c["B"]
+    if seq_len is not None:
+        if isinstance(c["L"], tuple):
+            raise ValueError(f"{name} has ragged lengths; seq_len applies to uniform-length workloads")
+        c["L"] = int(seq_len)
+        name = f"{name}_L{int(seq_len)}"
     if isinstance(c["L"], tuple):
         # ragged: lengths and per-sequence ART parameters come first in the draw order
         gen = torch.Generator().manual_seed(int(seed) ^ 0x5EED)
