@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import struct
 from typing import Optional
 
 import torch
@@ -63,6 +64,35 @@ class ArtParams(ctypes.Structure):
         ("workspace_bytes", ctypes.c_int64)]
 
 
+def _struct_format(cls) -> str:
+    """struct-module format of a ctypes Structure, padding included, read
+    from the structure's own field offsets (so it always matches art.h as the
+    ctypes declaration does)."""
+    codes = {ctypes.c_void_p: "Q", ctypes.c_int32: "i", ctypes.c_int64: "q", ctypes.c_float: "f"}
+    parts, off = [], 0
+    for name, ty in cls._fields_:
+        fo = getattr(cls, name).offset
+        if fo > off:
+            parts.append(f"{fo - off}x")
+            off = fo
+        if isinstance(ty, type) and issubclass(ty, ctypes.Structure):
+            parts.append(_struct_format(ty))
+        elif isinstance(ty, type) and issubclass(ty, ctypes.Array):
+            parts.append(f"{ty._length_}{codes[ty._type_]}")
+        else:
+            parts.append(codes.get(ty, "Q"))  # pointers are 8-byte addresses
+        off += ctypes.sizeof(ty)
+    if ctypes.sizeof(cls) > off:
+        parts.append(f"{ctypes.sizeof(cls) - off}x")
+    return "".join(parts)
+
+
+# art_params_t packed in one call: building the nested ctypes structures field
+# by field cost ~23 us of host time per call, packing them ~10 us
+_PARAMS = struct.Struct("<" + _struct_format(ArtParams))
+assert _PARAMS.size == ctypes.sizeof(ArtParams)
+
+
 _P = ctypes.POINTER
 _lib.art_decode_attention.argtypes = [_P(ArtTensor)] * 6 + [ctypes.c_float, ctypes.c_float, ctypes.c_int32,
                                                             ctypes.c_int32, _P(ArtTensor), _P(ArtTensor),
@@ -103,6 +133,22 @@ def art_version() -> int:
     return int(_lib.art_version())
 
 
+def _tensor_fields(t):
+    """The eleven art_tensor_t values of a tensor (all zero for None)."""
+    if t is None:
+        return (0,) * 11
+    n = t.dim()
+    sh, sd = tuple(t.shape), t.stride()
+    if n < 4:
+        pad = (0,) * (4 - n)
+        sh, sd = sh + pad, sd + pad
+    return (t.data_ptr() if t.numel() else 0, _DTYPE.get(t.dtype, -1), n) + sh + sd
+
+
+def _addr(t):
+    return t.data_ptr() if t is not None else 0
+
+
 def descriptor(t: torch.Tensor) -> ArtTensor:
     """art_tensor_t over a tensor's storage (no copy)."""
     d = ArtTensor()
@@ -121,8 +167,13 @@ def _need_cuda(*ts):
             raise ValueError("libart runs on the GPU only: every tensor must be on a CUDA device")
 
 
-def _stream(stream) -> Optional[int]:
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device=None) -> Optional[int]:
     if stream is None:
+        if _raw_stream is not None and device is not None and device.index is not None:
+            return _raw_stream(device.index)  # the same handle, without building a Stream object
         return torch.cuda.current_stream().cuda_stream
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -147,7 +198,7 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
           for t in (q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block)]
     refs = [ctypes.byref(x) if x is not None else None for x in ds]
     st = _lib.art_decode_attention(*refs[:6], float(eps_m), float(eps_d), int(P), int(min_blocks), refs[6],
-                                   refs[7], _stream(stream))
+                                   refs[7], _stream(stream, q.device))
     _check(st, "art_decode_attention")
     return out, stop_block
 
@@ -155,34 +206,25 @@ def art_decode_attention(q, k_cache, v_cache, page_table, block_order, seq_lens,
 def _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P, min_blocks,
             sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status,
             engine, cluster_size, stages, compute_warps, window, timeout_ns, debug_flags, prefetch, detector_off=0,
-            merge_cta=0):
+            merge_cta=0, want_info=True):
     """Fill art_params_t (argument marshalling only); returns (params, info)."""
     per = [eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq, blocks_fetched, device_status]
     _need_cuda(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, *per)
     for t, dt in zip(per, (torch.float32, torch.float32, torch.int32, torch.int32, torch.int32, torch.int32)):
         if t is not None and (t.dtype != dt or not t.is_contiguous()):
             raise ValueError(f"per-sequence/accounting arrays must be contiguous {dt}")
-    p = ArtParams()
-    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("page_table", page_table),
-                    ("block_order", block_order), ("seq_lens", seq_lens), ("out", out), ("stop_block", stop_block)):
-        if t is not None:           # block_order=None: the default order, built on the fly
-            setattr(p, name, descriptor(t))
-    p.eps_m, p.eps_d, p.P, p.min_blocks = float(eps_m), float(eps_d), int(P), int(min_blocks)
-    p.sm_scale = float(sm_scale)
-    p.eps_m_per_seq = eps_m_per_seq.data_ptr() if eps_m_per_seq is not None else None
-    p.eps_d_per_seq = eps_d_per_seq.data_ptr() if eps_d_per_seq is not None else None
-    p.P_per_seq = P_per_seq.data_ptr() if P_per_seq is not None else None
-    p.min_blocks_per_seq = min_blocks_per_seq.data_ptr() if min_blocks_per_seq is not None else None
-    p.blocks_fetched = blocks_fetched.data_ptr() if blocks_fetched is not None else None
-    p.device_status = device_status.data_ptr() if device_status is not None else None
-    p.engine, p.cluster_size, p.stages = int(engine), int(cluster_size), int(stages)
-    p.compute_warps, p.window, p.timeout_ns = int(compute_warps), int(window), int(timeout_ns)
-    p.debug_flags = int(debug_flags)
-    p.prefetch = int(prefetch)
-    p.detector_off = int(detector_off)
-    p.merge_cta = int(merge_cta)
-    info = ArtLaunchInfo()
-    p.info = ctypes.pointer(info)
+    p = ArtParams.from_buffer_copy(_PARAMS.pack(
+        *_tensor_fields(q), *_tensor_fields(k_cache), *_tensor_fields(v_cache), *_tensor_fields(page_table),
+        *_tensor_fields(block_order), *_tensor_fields(seq_lens), *_tensor_fields(out), *_tensor_fields(stop_block),
+        float(eps_m), float(eps_d), int(P), int(min_blocks), float(sm_scale),
+        _addr(eps_m_per_seq), _addr(eps_d_per_seq), _addr(P_per_seq), _addr(min_blocks_per_seq),
+        _addr(blocks_fetched), _addr(device_status), int(engine), int(cluster_size), int(stages),
+        int(compute_warps), int(window), int(timeout_ns), int(debug_flags), 0, int(prefetch), int(detector_off),
+        int(merge_cta), 0, 0))
+    info = None
+    if want_info:
+        info = ArtLaunchInfo()
+        p.info = ctypes.pointer(info)
     return p, info
 
 
@@ -204,12 +246,12 @@ def art_decode_attention_ex(q, k_cache, v_cache, page_table, block_order, seq_le
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta)
+                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta, want_info=want_info)
     if workspace is not None:
         _need_cuda(workspace)
         p.workspace = workspace.data_ptr()
         p.workspace_bytes = workspace.numel() * workspace.element_size()
-    st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream))
+    st = _lib.art_decode_attention_ex(ctypes.byref(p), _stream(stream, q.device))
     _check(st, "art_decode_attention_ex")
     if want_info:
         return out, stop_block, info.as_dict()
@@ -233,8 +275,8 @@ def art_decode_attention_multi(q, k_cache, v_cache, page_table, block_order, seq
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta)
-    st = _lib.art_decode_attention_multi(ctypes.byref(p), int(T), _stream(stream))
+                      timeout_ns, debug_flags, prefetch, detector_off, merge_cta, want_info=want_info)
+    st = _lib.art_decode_attention_multi(ctypes.byref(p), int(T), _stream(stream, q.device))
     _check(st, "art_decode_attention_multi")
     if want_info:
         return out, stop_block, info.as_dict()
@@ -256,7 +298,7 @@ def art_workspace_bytes(q, k_cache, v_cache, page_table, block_order, seq_lens, 
               cluster_size=0, stages=0, compute_warps=0, window=0, timeout_ns=0, debug_flags=0, prefetch=0,
               detector_off=0, merge_cta=0)
     kw.update(options)
-    p, _ = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, **kw)
+    p, _ = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, want_info=False, **kw)
     n = int(_lib.art_workspace_bytes(ctypes.byref(p)))
     if n < 0:
         raise ArtError(n, "art_workspace_bytes")
@@ -281,8 +323,8 @@ def art_decode_attention_no_alloc(q, k_cache, v_cache, page_table, block_order, 
     p, info = _params(q, k_cache, v_cache, page_table, block_order, seq_lens, out, stop_block, eps_m, eps_d, P,
                       min_blocks, sm_scale, eps_m_per_seq, eps_d_per_seq, P_per_seq, min_blocks_per_seq,
                       blocks_fetched, device_status, engine, cluster_size, stages, compute_warps, window,
-                      timeout_ns, 0, prefetch, detector_off, 0)
-    st = _lib.art_decode_attention_no_alloc(ctypes.byref(p), _stream(stream))
+                      timeout_ns, 0, prefetch, detector_off, 0, want_info=want_info)
+    st = _lib.art_decode_attention_no_alloc(ctypes.byref(p), _stream(stream, q.device))
     _check(st, "art_decode_attention_no_alloc")
     if want_info:
         return out, stop_block, info.as_dict()

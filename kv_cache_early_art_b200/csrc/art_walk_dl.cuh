@@ -187,6 +187,14 @@ __device__ void share_role_dl(const KernelArgs &a, const Shared &sh, int N, cons
         const float *spk = sh.ring + (size_t)sk * slot_floats;
         uint64_t t0 = 0;
         for (uint32_t it = 0; !quit; ++it) {
+            // Once the final decision is in, the batch may never come, and a
+            // try_wait on a phase that never completes suspends the warp until
+            // the hardware's time limit: the final word is read before every
+            // poll, so the warp leaves after at most one such suspension.
+            if (__shfl_sync(0xffffffffu, lane == 0 && ctl[3] != kDLNone ? 1 : 0, 0)) {
+                quit = 2;
+                break;
+            }
             const bool arrived = lane < nmax && mbar_try_wait(sh.ready(sk), pk);
             if (__any_sync(0xffffffffu, arrived && __float_as_uint(spk[0]) != 0u)) {
                 quit = 1;
@@ -202,8 +210,6 @@ __device__ void share_role_dl(const KernelArgs &a, const Shared &sh, int N, cons
                         t0 = now;
                     if (*sh.abort) {
                         q = 1;
-                    } else if (ctl[3] != kDLNone) {
-                        q = 2;
                     } else if ((int64_t)(now - t0) > a.timeout_ns) {
                         *sh.abort = 1u;
                         record_error(a.device_status, kErrTimeout);

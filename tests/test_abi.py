@@ -266,3 +266,47 @@ def test_multi_query_host_errors(art):
     p = multi_params(art)
     p.k_cache.dtype = 0
     assert r(p) == -3                                         # cache dtype differs from q
+
+
+def test_packed_params_equal_field_by_field(art):
+    """The binding packs art_params_t in one struct call; the bytes must be
+    those of the same structure filled field by field through ctypes, for
+    every tensor rank the entry points take and for every option."""
+    import torch
+    from kv_cache_early_art_b200 import binding as B
+    g = torch.Generator().manual_seed(5)
+    q = torch.zeros(3, 8, 128, dtype=torch.bfloat16)[:, :, :]
+    k = torch.zeros(20, 2, 64, 128, dtype=torch.bfloat16)
+    v = torch.zeros(20, 2, 64, 128, dtype=torch.bfloat16).transpose(0, 1).contiguous().transpose(0, 1)
+    pt = torch.zeros(3, 7, dtype=torch.int32)
+    bo = torch.zeros(3, 7, dtype=torch.int32)
+    sl = torch.zeros(3, dtype=torch.int32)
+    out = torch.zeros(3, 8, 128)
+    st = torch.zeros(3, 2, dtype=torch.int32)
+    em = torch.zeros(3)
+    orig = B._need_cuda
+    B._need_cuda = lambda *a: None
+    try:
+        for trial in range(6):
+            opts = [int(x) for x in torch.randint(0, 9, (11,), generator=g)]
+            args = (q, k, v, pt, bo if trial % 2 else None, sl, out, st, 1e-3 * trial, 2e-4, opts[0], opts[1],
+                    0.25 * trial, em, None if trial % 3 else em, sl, None, sl if trial > 2 else None, sl, opts[2],
+                    opts[3], opts[4], opts[5], opts[6], 12345678901 * trial, opts[7] % 2, opts[8], opts[9] % 2,
+                    opts[10] % 3 - 1)
+            p, _ = B._params(*args, want_info=False)
+            ref = B.ArtParams()
+            for name, t in zip(("q", "k_cache", "v_cache", "page_table", "block_order", "seq_lens", "out",
+                                "stop_block"), args[:8]):
+                if t is not None:
+                    setattr(ref, name, B.descriptor(t))
+            for name, val in zip(("eps_m", "eps_d", "P", "min_blocks", "sm_scale"), args[8:13]):
+                setattr(ref, name, val)
+            for name, t in zip(("eps_m_per_seq", "eps_d_per_seq", "P_per_seq", "min_blocks_per_seq",
+                                "blocks_fetched", "device_status"), args[13:19]):
+                setattr(ref, name, t.data_ptr() if t is not None else None)
+            for name, val in zip(("engine", "cluster_size", "stages", "compute_warps", "window", "timeout_ns",
+                                  "debug_flags", "prefetch", "detector_off", "merge_cta"), args[19:]):
+                setattr(ref, name, val)
+            assert bytes(p) == bytes(ref), trial
+    finally:
+        B._need_cuda = orig
