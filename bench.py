@@ -423,6 +423,7 @@ def run_ours(args):
             "hbm_frac_of_measured": fetch_bytes / (ms_walk / 1000.0) / 1e9 / peak,
             "hbm_frac_of_8tbs_spec": fetch_bytes / (ms_walk / 1000.0) / 1e9 / SPEC_HBM_GBS,
             "skip_frac_blocks": 1.0 - consumed / full_blocks,
+            "skip_frac_bytes": 1.0 - fetched_blocks / full_blocks,   # the pages never read (speculation counted)
             "fetch_waste_blocks": fetched_blocks - consumed,
             "walk_ms": ms_walk,
             "full_attention": {"walk_ms": ms_full, "kv_gbs": full_consumed * block_bytes / (ms_full / 1000.0) / 1e9,
