@@ -272,7 +272,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_for(args.workload, w, args.gpus),
+            "config": dict(config_for(args.workload, w, args.gpus),
+                           l2="not applicable: the oracle runs on the host cores"),
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": ncores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
