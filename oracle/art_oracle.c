@@ -8,11 +8,11 @@
  * Large Language Model Decoding" (gist.science explainer), Technical Summary
  * section 2 -- 2.1 streaming tile-wise accumulation of the attention output,
  * 2.2 the two stability statistics and their thresholds, 2.3 the patience
- * counter, 2.4 traversal reordering and the mandatory sink block.  The exact
- * statistic formulas are the task specification's (full-vector relative
- * magnitude change and one minus cosine, both strict "<"); the explainer
- * words them as "L2-norm difference" and "cosine similarity deviation" of a
- * probe vector.
+ * counter, 2.4 traversal reordering and the mandatory sink block.  The
+ * statistics used here are the full-vector relative magnitude change and one
+ * minus the cosine, both compared with a strict "<"; the explainer words
+ * them as "L2-norm difference" and "cosine similarity deviation" of a probe
+ * vector.
  *
  * Arithmetic: every input value is upcast exactly to double; all sums,
  * exponentials and statistics are double precision; no blocking, fusion or

@@ -1,7 +1,7 @@
 """GPU parity for the ablation modes (ART explainer, Technical Summary §4:
 removing the scale or the direction criterion, or the patience mechanism),
-the undecided band around a threshold (§2.2 thresholds, the task's 1e-4
-relative band), and launch-option and length edge cases."""
+the undecided band around a threshold (§2.2 thresholds; the acceptance
+rule's 1e-4 relative band), and launch-option and length edge cases."""
 import numpy as np
 import pytest
 import torch
