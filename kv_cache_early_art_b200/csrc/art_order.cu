@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 2 ? 4 : 2) art_block_score_ker
 // Wide summaries (more than four vectors per lane): the group sums of the
 // query rows sit in shared memory, filled by the whole CTA first.
 template <typename TQ, typename TS, int CH>
-__global__ void __launch_bounds__(kThreads) art_block_score_wide_kernel(ScoreArgs a)
+__global__ void __launch_bounds__(kThreads, 2) art_block_score_wide_kernel(ScoreArgs a)
 {
     // CH: summary vectors per lane and block kept in flight (1, 2 or 4)
     extern __shared__ float qg[];   // [Hkv * d]: sum of the group's query heads
