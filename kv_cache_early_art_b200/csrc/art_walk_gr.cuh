@@ -91,6 +91,12 @@ __device__ void share_role_gr(const KernelArgs &a, const Shared &sh, int unit, i
         uint64_t t0 = 0;
         bool landed_b = false;
         for (uint32_t it = 0; !quit; ++it) {
+            // once the final decision is in, the remaining states never come:
+            // the word is read on every pass (a pass waits on global loads)
+            if (__shfl_sync(0xffffffffu, lane == 0 && ctl[3] != kDLNone ? 1 : 0, 0)) {
+                quit = 2;
+                break;
+            }
             if (mine && !issued) {
                 const unsigned long long v = ld_acquire_gpu_u64(gfl + jk % a.Rg);
                 if (v == (ep | (unsigned long long)(jk + 1))) {
@@ -129,8 +135,6 @@ __device__ void share_role_gr(const KernelArgs &a, const Shared &sh, int unit, i
                         t0 = now;
                     if (*sh.abort) {
                         q = 1;
-                    } else if (ctl[3] != kDLNone) {
-                        q = 2;
                     } else if ((int64_t)(now - t0) > a.timeout_ns) {
                         *sh.abort = 1u;
                         record_error(a.device_status, kErrTimeout);
