@@ -60,3 +60,19 @@ def test_oracle_sample_is_bounded():
     assert used == 3 and done >= 2 and qps > 0
     g = bench.sequences(w, [1, 3])
     assert g.B == 2 and g.seq_lens.tolist() == [9, 1]
+
+
+def test_seq_len_override_keeps_the_shape():
+    """bench.py --seq-len builds a smaller case of the same workload (for
+    profiling): the same batch, heads, page size and parameters, the new
+    length, its own name; a ragged workload refuses it."""
+    import pytest
+    from kv_cache_early_art_b200.workloads import make_workload
+    w = make_workload("tiny_fp32")
+    s = make_workload("tiny_fp32", seq_len=256)
+    assert (s.B, s.Hq, s.Hkv, s.d, s.page) == (w.B, w.Hq, w.Hkv, w.d, w.page)
+    assert s.name == "tiny_fp32_L256" and int(s.seq_lens.max()) == 256
+    assert int(s.n_blocks().max()) == 256 // s.page
+    assert w.uniform_params() == s.uniform_params()
+    with pytest.raises(ValueError):
+        make_workload("mistral7b_b128", seq_len=1024)
