@@ -209,21 +209,39 @@ def test_workspace_size_rules(cuda_lib):
     assert cuda_lib.art_workspace_bytes(wm.q, wm.k_cache, wm.v_cache, wm.page_table, None, wm.seq_lens) == 0
 
 
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("G", [4, 8])
-def test_single_unit_largest_cluster(cuda_lib, G):
+def test_single_unit_largest_cluster(cuda_lib, G, mode):
     """One (sequence, kv-head) unit: the automatic launch gives the dedicated
-    merge CTA the largest cluster that fits (sixteen CTAs, fifteen fetching).
-    A long sequence with planted keys stops mid-way; the same cache at eps = 0
-    is full attention.  Both against the oracle."""
+    merge CTA the largest cluster that fits (sixteen CTAs, fifteen fetching),
+    or, through a workspace, every other CTA of the GPU.  A long sequence with
+    planted keys stops mid-way; the same cache at eps = 0 is full attention.
+    Both against the oracle."""
     L = 64 * 700 + 23
     w = make_custom(B=1, Hq=G, Hkv=1, d=128, page=64, dtype="bf16", seq_lens=[L], seed=970 + G, keys="recency",
                     planted=3, planted_gain=5.0, order="random", eps_m=2e-3, eps_d=2e-4, P=3, min_blocks=2)
-    out, stop, fetched, status, info = run_gpu(cuda_lib, w)
-    assert status == 0 and info["merge_cta"] == 1 and info["cluster_size"] >= 8
+    kw = {} if mode == "cluster" else mode_kw(cuda_lib, w, mode)
+    out, stop, fetched, status, info = run_gpu(cuda_lib, w, **kw)
+    assert status == 0 and info["merge_cta"] == (1 if mode == "cluster" else 2) and info["cluster_size"] >= 8
     parity.check(w, out, stop)
     assert_fetch_bound(w, stop, fetched, info["window"])
     w0 = w.to("cpu")
     w0.eps_m, w0.eps_d = torch.zeros(1), torch.zeros(1)
-    out0, stop0, fetched0, status0, info0 = run_gpu(cuda_lib, w0)
+    out0, stop0, fetched0, status0, info0 = run_gpu(cuda_lib, w0, **kw)
     assert status0 == 0 and int(stop0.item()) == int(w.n_blocks()[0])
     parity.check(w0, out0, stop0)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_short_units_largest_cluster(cuda_lib, mode):
+    """Very short sequences (1 to 9 blocks) on the largest clusters: most
+    fetching CTAs get no block at all; stops and outputs as the oracle's."""
+    lens = [1, 64, 65, 64 * 3 + 1, 64 * 5, 64 * 9 - 7]
+    w = make_custom(B=len(lens), Hq=8, Hkv=1, d=128, page=64, dtype="bf16", seq_lens=lens, seed=975,
+                    keys="recency", planted=1, planted_gain=4.0, order="random", eps_m=5e-3, eps_d=5e-4, P=1,
+                    min_blocks=1)
+    kw = {} if mode == "cluster" else mode_kw(cuda_lib, w, mode)
+    out, stop, fetched, status, info = run_gpu(cuda_lib, w, **kw)
+    assert status == 0 and info["merge_cta"] == (1 if mode == "cluster" else 2)
+    parity.check(w, out, stop)
+    assert_fetch_bound(w, stop, fetched, info["window"])
