@@ -189,7 +189,10 @@ typedef struct {
                                    /* (block states, ready tags and counters; at least      */
                                    /* art_workspace_bytes(p) bytes, 256-byte aligned).  It  */
                                    /* needs no clearing: every word is tagged with the      */
-                                   /* call.  Calls that overlap on the GPU must not share   */
+                                   /* call (a 32-bit count of this process's calls, so a    */
+                                   /* word left untouched for 2^32 calls could read as      */
+                                   /* current: clear a workspace idle that long before      */
+                                   /* reuse).  Calls that overlap on the GPU must not share */
                                    /* one workspace.                                        */
     int64_t workspace_bytes;       /* its size                                              */
 } art_params_t;
@@ -242,7 +245,10 @@ int64_t art_workspace_bytes(const art_params_t *p);
  * device current and keeps it; make that first call before any stream capture
  * begins.  Every call on a device shares the one array and it keeps what the
  * last call left; nothing in it needs clearing, since each control word the
- * walk reads is tagged with the call that wrote it.  Calls whose kernels
+ * walk reads is tagged with the call that wrote it (a 32-bit count of the
+ * process's calls: a word no call has rewritten for 2^32 calls could read as
+ * current, which needs problems whose units shrink and then grow again across
+ * that many calls).  Calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on the array:
  * order them on one stream or serialise them.
  */
